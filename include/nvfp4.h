@@ -1,0 +1,238 @@
+/*
+ * nvfp4.h — C ABI of libnvfp4: NVFP4 activation quantization, the W4A4
+ * block-scaled GEMM and the NVFP4 KV cache, for one sm_100a GPU.
+ *
+ * Sources (web pages describing LongLive-2.0; cited by title and section):
+ *   [TW]  techwalker.com, "NVIDIA研究团队打造全球首个FP4视频生成系统，速度提升两倍还省一半内存"
+ *         §一 "给AI视频生成做一次'瘦身手术'"  — the NVFP4 format: 4-bit E2M1 values,
+ *             one FP8 scale per 16 values, one FP32 scale for the whole tensor.
+ *         §三 "让视频一段一段'流水线式'地生成" — generation proceeds chunk by chunk
+ *             (8 frames per chunk), each chunk appended to the KV cache.
+ *         §四 "推理时三把'加速钥匙'" — all matmuls run in 4-bit (W4A4); the KV cache
+ *             is stored in NVFP4 after subtracting the mean of K; a parallel CUDA
+ *             kernel dequantizes several cache chunks of one window at once.
+ *   [ZD]  github.zuobiaodaohang.com, "长视频生成的两堵物理墙" (NVlabs/LongLive write-up),
+ *         section "NVFP4：数据体积砍到 1/4，带宽压力降一个数量级" — weights, activations
+ *         and KV cache all 4-bit; the quantized KV cache is updated in place.
+ *   [RM]  news.ainew.jp copy of the LongLive 2.0 README, "Quick Start / NVFP4" —
+ *         weights are materialized once in NVFP4; quantized buffers must never be
+ *         dtype-cast (so they cross this ABI as raw bytes).
+ *
+ * Number format (the readings this library fixes where the pages are silent):
+ *   E2M1 code: bit 3 = sign, bits 0..2 index the magnitudes {0,0.5,1,1.5,2,3,4,6}.
+ *   E4M3 block scale: OCP E4M3FN (bias 7, max 448, no Inf), one byte per 16
+ *     consecutive values of a row, never negative, never NaN.
+ *   Tensor scale g = RN_f32(amax / 2688), 2688 = 6 * 448, amax = max |x|.
+ *   Block scale s = E4M3_RNE_satfinite(RN_f32(amax_block / RN_f32(6 * g))).
+ *   Element code = sign(x) | E2M1 round-to-nearest-even of the EXACT quotient
+ *     |x| / D with D = RN_f32(s * g), saturating at 6.  D == 0 gives magnitude 0.
+ *   Decoded value = RN_f32(RN_f32(e2m1 * s) * g).
+ *   Packing: element 2i of a row in the low nibble of byte i, 2i+1 in the high nibble.
+ *
+ * Conventions for every entry point:
+ *   - All tensor pointers are DEVICE pointers owned by the caller; the library
+ *     never allocates or frees device memory inside these calls.
+ *   - Work is enqueued on `stream` (a cudaStream_t; NULL = legacy default stream)
+ *     and runs asynchronously.  Argument errors are detected on the host, return
+ *     a status and enqueue nothing.
+ *   - Data errors found on the device (a NaN/Inf input, a wait that gave up)
+ *     set a sticky per-device status word (read it with nvfp4_get_device_status);
+ *     the affected kernel then writes no output.  No kernel ever traps.
+ *   - A device that is not compute capability 10.0 returns
+ *     NVFP4_ERR_UNSUPPORTED_DEVICE.  There is no fallback path.
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t; declared here so this header needs no CUDA headers. */
+typedef struct CUstream_st* nvfp4_stream_t;
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,        /* NULL pointer, bad enum, bad slot, overlap   */
+  NVFP4_ERR_SHAPE = 2,              /* dimension mismatch or unsupported size      */
+  NVFP4_ERR_ALIGNMENT = 3,          /* pointer or leading dimension misaligned     */
+  NVFP4_ERR_NONFINITE = 4,          /* device status: a NaN or Inf input value     */
+  NVFP4_ERR_TIMEOUT = 5,            /* device status: a bounded wait gave up       */
+  NVFP4_ERR_CUDA = 6,               /* a CUDA runtime call failed                  */
+  NVFP4_ERR_UNSUPPORTED_DEVICE = 7  /* current device is not sm_100                */
+} nvfp4_status;
+
+typedef enum { NVFP4_BF16 = 0, NVFP4_FP32 = 1 } nvfp4_dtype;
+
+/* Layout of the E4M3 block scales of an nvfp4_tensor.
+ *   NVFP4_SF_ROWMAJOR: byte (r, j) at scales[r * ld_scales + j], j < cols/16.
+ *   NVFP4_SF_MMA: the tensor-core operand layout.  Rows are grouped in tiles of
+ *     128 and block-scale columns in groups of 4 (64 values of the row); each
+ *     (row-tile, group) pair is one 512-byte atom, atoms stored row-tile-major:
+ *       atom  = (r / 128) * ceil(cols / 64) + (j / 4)
+ *       byte  = atom * 512 + (r % 32) * 16 + ((r % 128) / 32) * 4 + (j % 4)
+ *     Total size nvfp4_scales_bytes(rows, cols, NVFP4_SF_MMA); padding bytes
+ *     (rows beyond `rows`, groups beyond cols/16) are written as 0 by the
+ *     library and must stay 0.  ld_scales is ignored.
+ */
+typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA = 1 } nvfp4_sf_layout;
+
+/* One NVFP4 tensor [rows, cols] (cols % 16 == 0), all device memory:
+ *   codes : rows * ld_codes bytes; ld_codes >= cols / 2, multiple of 16;
+ *           base 16-byte aligned.
+ *   scales: see nvfp4_sf_layout; base 16-byte aligned.
+ *   gscale: one FP32 tensor scale g. */
+typedef struct nvfp4_tensor {
+  uint8_t* codes;
+  uint8_t* scales;
+  float* gscale;
+  int64_t rows;
+  int64_t cols;
+  int64_t ld_codes;
+  int64_t ld_scales;
+  int32_t sf_layout; /* nvfp4_sf_layout */
+  int32_t reserved;  /* must be 0 */
+} nvfp4_tensor;
+
+/* Bytes of the scale array of a [rows, cols] tensor in the given layout
+ * (ROWMAJOR assumes ld_scales = cols / 16). */
+nvfp4_status nvfp4_scales_bytes(int64_t rows, int64_t cols, int32_t sf_layout, size_t* bytes);
+
+/* nvfp4_quantize — activation (or weight) quantization to NVFP4.
+ * [TW] §一 defines the format; [TW] §四 / [ZD] apply it to activations and weights.
+ *   x        : device, row-major [rows, cols] of `xt` (NVFP4_BF16 or NVFP4_FP32),
+ *              leading dimension ldx elements (ldx >= cols); base and row pitch
+ *              16-byte aligned.
+ *   gscale_in: NULL  -> the tensor scale is computed from x: g = RN(amax / 2688)
+ *                       (two passes over x). amax_out is then REQUIRED.
+ *              !NULL -> device FP32 g used as given (one pass over x, e.g. a
+ *                       scale calibrated on an earlier chunk).
+ *   out      : rows/cols must match; codes, scales, gscale written; *out->gscale
+ *              receives the g that was used.
+ *   amax_out : device FP32, receives max|x| (nullable when gscale_in != NULL).
+ * Errors: INVALID_ARG (NULL, bad dtype/layout), SHAPE (cols % 16, rows/cols
+ * mismatch, ldx < cols), ALIGNMENT; device status NONFINITE if x holds NaN/Inf
+ * (then nothing is written except amax_out). */
+nvfp4_status nvfp4_quantize(const void* x, int32_t xt, int64_t rows, int64_t cols, int64_t ldx,
+                            const float* gscale_in, const nvfp4_tensor* out, float* amax_out,
+                            nvfp4_stream_t stream);
+
+/* nvfp4_dequantize — y = RN(RN(e2m1 * s) * g), stored as FP32 or as bf16 (RNE).
+ * [TW] §一 (format).  y: device row-major [rows, cols], leading dimension ldy
+ * elements, 16-byte aligned base and row pitch.  Either scale layout. */
+nvfp4_status nvfp4_dequantize(const nvfp4_tensor* in, void* y, int32_t yt, int64_t ldy,
+                              nvfp4_stream_t stream);
+
+typedef enum { NVFP4_ACT_NONE = 0, NVFP4_ACT_GELU_TANH = 1 } nvfp4_activation;
+
+/* Optional GEMM epilogue.
+ *   act         : NVFP4_ACT_NONE or NVFP4_ACT_GELU_TANH,
+ *                 h = 0.5 c (1 + tanh(sqrt(2/pi) (c + 0.044715 c^3))) in FP32.
+ *   q_out       : non-NULL -> h is quantized to NVFP4 inside the GEMM (blocks of 16
+ *                 along N) into q_out ([M, N], NVFP4_SF_MMA so that it can feed the
+ *                 next GEMM as its A operand).  [AM] "scaling and quantization fused
+ *                 into one kernel"; the tensor scale cannot be known before the
+ *                 GEMM ends, so it is SUPPLIED:
+ *   q_gscale_in : device FP32 g used for q_out (required with q_out; copied to
+ *                 *q_out->gscale).
+ *   q_amax_out  : device FP32, nullable: receives max|h| (calibrates the next call).
+ *   h_out       : device FP32 [M, N] (ld = N), nullable: also store h (verification).
+ */
+typedef struct nvfp4_epilogue {
+  int32_t act;
+  int32_t reserved;
+  const nvfp4_tensor* q_out;
+  const float* q_gscale_in;
+  float* q_amax_out;
+  float* h_out;
+} nvfp4_epilogue;
+
+/* nvfp4_gemm — C[m, n] = RN(acc[m, n] * RN(gA * gW)) with
+ * acc = sum_k (e2m1(A) sA)(e2m1(W) sW) accumulated in FP32 by the tensor cores.
+ * [TW] §四: the linear layers are the dominant cost and all run in 4-bit.
+ *   A : [M, K] NVFP4, W : [N, K] NVFP4 (both K-major, i.e. row-major, both with
+ *       sf_layout NVFP4_SF_MMA).  K % 64 == 0 is not required (the scale padding
+ *       of the MMA layout is zero), K % 32 == 0 is (row pitch of codes).
+ *   C : device row-major [M, N] of ct (FP32 or bf16), leading dimension ldc
+ *       elements; may be NULL when ep->q_out is set.
+ *   ep: nullable epilogue (activation, fused requantization).
+ * Requires N % 16 == 0.  Errors: INVALID_ARG, SHAPE, ALIGNMENT; device status
+ * TIMEOUT if a pipeline wait gave up. */
+nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, int32_t ct,
+                        int64_t ldc, const nvfp4_epilogue* ep, nvfp4_stream_t stream);
+
+/* ---------------------------------------------------------------- KV cache ----
+ * [TW] §四: K has its mean subtracted, then K and V are stored in NVFP4 (about
+ * 1.125 bytes per K+V element pair vs 4 in bf16).  [TW] §三: chunks of tokens are
+ * appended one by one; [ZD]: the cache is updated in place.
+ * Reading fixed here: the mean mu is per (head, dim) over the chunk's tokens,
+ *   mu = RN_f32(exact_sum / tokens), kept in FP32 and added back on dequant;
+ *   K' = RN_f32(k - mu); one tensor scale per chunk for K' and one for V;
+ *   16-value blocks run along head_dim.
+ * Device layout of one cache (all inside the caller's allocation):
+ *   k_codes [max_chunks][chunk_tokens][heads][head_dim/2]   (same for v_codes)
+ *   k_scales[max_chunks][chunk_tokens][heads][head_dim/16]  (same for v_scales)
+ *   mu      [max_chunks][heads][head_dim] FP32
+ *   gscale  [max_chunks][2] FP32 (g_K, g_V)
+ *   scratch used by kv_quant_append (per-column statistics of one chunk).
+ */
+typedef struct nvfp4_kv_cache {
+  uint8_t* base;          /* device allocation given to nvfp4_kv_cache_init */
+  size_t bytes;
+  int32_t heads;
+  int32_t head_dim;       /* multiple of 16 */
+  int64_t chunk_tokens;
+  int32_t max_chunks;
+  int32_t reserved;
+  int64_t off_k_codes, off_v_codes, off_k_scales, off_v_scales;
+  int64_t off_mu, off_gscale, off_scratch;
+  int64_t slot_codes_bytes;   /* chunk_tokens * heads * head_dim / 2  */
+  int64_t slot_scales_bytes;  /* chunk_tokens * heads * head_dim / 16 */
+} nvfp4_kv_cache;
+
+/* Device bytes needed by a cache of the given geometry. */
+nvfp4_status nvfp4_kv_cache_bytes(int32_t heads, int32_t head_dim, int64_t chunk_tokens,
+                                  int32_t max_chunks, size_t* bytes);
+
+/* Lays out a cache in caller-owned device memory `dev_mem` (256-byte aligned,
+ * `bytes` >= nvfp4_kv_cache_bytes(...)) and fills the host struct `cache`.
+ * No device work is enqueued; slots hold garbage until appended. */
+nvfp4_status nvfp4_kv_cache_init(void* dev_mem, size_t bytes, int32_t heads, int32_t head_dim,
+                                 int64_t chunk_tokens, int32_t max_chunks, nvfp4_kv_cache* cache);
+
+/* kv_quant_append — quantize one chunk of K and V into slot `slot`, in place.
+ *   k, v   : device bf16 [tokens][heads][head_dim], 16-byte aligned.
+ *   tokens : must equal cache->chunk_tokens.
+ * Appends to one cache must be issued on one stream (they share the scratch).
+ * Device status NONFINITE on NaN/Inf input (the slot is then left unchanged). */
+nvfp4_status kv_quant_append(const nvfp4_kv_cache* cache, const void* k, const void* v,
+                             int64_t tokens, int32_t slot, nvfp4_stream_t stream);
+
+/* kv_dequant_window — dequantize the chunks listed in `slots_host` (a HOST array
+ * of n_slots slot ids, 1 <= n_slots <= 64, repeats allowed, any order) in one
+ * launch, writing bf16 [n_slots * chunk_tokens][heads][head_dim] to k_out and
+ * v_out (device, 16-byte aligned) in list order:
+ *   K^ = bf16(RN(RN(RN(e2m1 * s) * g_K) + mu)),  V^ = bf16(RN(RN(e2m1 * s) * g_V)). */
+nvfp4_status kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t* slots_host,
+                               int32_t n_slots, void* k_out, void* v_out,
+                               nvfp4_stream_t stream);
+
+/* ----------------------------------------------------------------- status ----
+ * Reads the sticky device status word of CUDA device `device` (synchronizes that
+ * device first).  *status_out is NVFP4_OK or the first data error recorded since
+ * the last clear; clear != 0 resets it to NVFP4_OK. */
+nvfp4_status nvfp4_get_device_status(int32_t device, int32_t* status_out, int32_t clear);
+
+/* Human-readable name of a status code (static string). */
+const char* nvfp4_status_string(int32_t status);
+
+/* Library version, (major << 16) | minor. */
+int32_t nvfp4_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* NVFP4_H_ */
