@@ -150,14 +150,15 @@ typedef struct nvfp4_epilogue {
   float* h_out;
 } nvfp4_epilogue;
 
-/* nvfp4_gemm — C[m, n] = RN(acc[m, n] * RN(gA * gW)) with
+/* nvfp4_gemm — C[m, n] = act(RN(acc[m, n] * RN(gA * gW))) with
  * acc = sum_k (e2m1(A) sA)(e2m1(W) sW) accumulated in FP32 by the tensor cores.
  * [TW] §四: the linear layers are the dominant cost and all run in 4-bit.
  *   A : [M, K] NVFP4, W : [N, K] NVFP4 (both K-major, i.e. row-major, both with
  *       sf_layout NVFP4_SF_MMA).  K % 64 == 0 is not required (the scale padding
  *       of the MMA layout is zero), K % 32 == 0 is (row pitch of codes).
  *   C : device row-major [M, N] of ct (FP32 or bf16), leading dimension ldc
- *       elements; may be NULL when ep->q_out is set.
+ *       elements; may be NULL when the epilogue writes another output (q_out,
+ *       h_out or q_amax_out).
  *   ep: nullable epilogue (activation, fused requantization).
  * Requires N % 16 == 0.  Errors: INVALID_ARG, SHAPE, ALIGNMENT; device status
  * TIMEOUT if a pipeline wait gave up. */

@@ -1,0 +1,216 @@
+// common.cuh — device helpers shared by the libnvfp4 kernels (sm_100a).
+//
+// Number format, as fixed by the library (techwalker.com, "NVIDIA研究团队打造全球首个FP4视频
+// 生成系统，速度提升两倍还省一半内存", §一: 4-bit E2M1 values, one FP8 scale per 16 values,
+// one FP32 scale for the whole tensor):
+//   g  = RN(amax / 2688)                       tensor scale (2688 = 6 * 448)
+//   s  = E4M3_RNE_sat(RN(amax_b / RN(6 g)))    block scale, one byte per 16 values
+//   D  = RN(value(s) * g)
+//   code = sign(x) | E2M1 round-to-nearest-even of the exact quotient |x| / D
+// All arithmetic here is IEEE binary32 round-to-nearest-even; the library is
+// compiled with -fmad=false so no product/sum pair is silently fused, and every
+// intended fused multiply-add is written as fmaf().
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nvfp4 {
+
+enum : unsigned { kStatusOk = 0, kStatusNonfinite = 4, kStatusTimeout = 5 };
+
+// The first data error wins; later ones leave the word unchanged (sticky).
+__device__ __forceinline__ void set_status(unsigned* status, unsigned code) {
+  atomicCAS(status, 0u, code);
+}
+
+// ---------------------------------------------------------------- loads/stores
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+__device__ __forceinline__ void stg_v4(void* p, uint4 v) {
+  asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" ::"l"(p), "r"(v.x), "r"(v.y), "r"(v.z),
+               "r"(v.w)
+               : "memory");
+}
+
+__device__ __forceinline__ void stg_v2(void* p, uint2 v) {
+  asm volatile("st.global.v2.u32 [%0], {%1,%2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
+}
+
+// ---------------------------------------------------------------- bf16 / fp32
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// two floats -> packed bf16x2 (RNE); `lo` lands in the low half
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
+// ---------------------------------------------------------------- E4M3
+// RNE with saturation to 448 of a finite s >= 0 (hardware conversion).
+__device__ __forceinline__ uint32_t e4m3_from_float(float s) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(s));
+  return (uint32_t)(r & 0xFFu);
+}
+
+// Value of a non-negative E4M3 byte (never NaN here): exponent field 0 is the
+// subnormal range m * 2^-9; otherwise the fields map straight onto binary32.
+__device__ __forceinline__ float e4m3_to_float(uint32_t b) {
+  const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
+  const float normal = __uint_as_float(((b & 0x7Fu) << 20) + (120u << 23));
+  const float sub = __int2float_rn((int)m) * 0.001953125f;  // exact
+  return e ? normal : sub;
+}
+
+// ---------------------------------------------------------------- E2M1
+// Exact E2M1 magnitude index of |x| / D by comparing |x| with each midpoint
+// m * D (m = 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5).  fmaf gives the correctly
+// rounded |x| - m D, whose sign is exact whenever D >= 2^-100 (the difference is
+// then either 0 or far above the binary32 underflow threshold).  A tie counts
+// toward the even neighbour: "> 0" where the lower index is even, ">= 0" where
+// the upper one is.
+__device__ __forceinline__ uint32_t e2m1_index_exact(float ax, float D) {
+  uint32_t i = 0;
+  i += fmaf(-0.25f, D, ax) > 0.0f;
+  i += fmaf(-0.75f, D, ax) >= 0.0f;
+  i += fmaf(-1.25f, D, ax) > 0.0f;
+  i += fmaf(-1.75f, D, ax) >= 0.0f;
+  i += fmaf(-2.5f, D, ax) > 0.0f;
+  i += fmaf(-3.5f, D, ax) >= 0.0f;
+  i += fmaf(-5.0f, D, ax) > 0.0f;
+  return i;
+}
+
+// Same decision in double for tiny D (every m * D is exact in double).
+static __device__ __noinline__ uint32_t e2m1_index_exact_f64(float ax, float D) {
+  const double a = ax, d = D;
+  uint32_t i = 0;
+  i += a > 0.25 * d;
+  i += a >= 0.75 * d;
+  i += a > 1.25 * d;
+  i += a >= 1.75 * d;
+  i += a > 2.5 * d;
+  i += a >= 3.5 * d;
+  i += a > 5.0 * d;
+  return i;
+}
+
+// Hardware RNE of two floats onto E2M1 (saturating at 6): `lo` in bits 0..3.
+__device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
+      "cvt.u32.u8 %0, t;\n\t}"
+      : "=r"(r)
+      : "f"(hi), "f"(lo));
+  return r;
+}
+
+// Block encoder: D = RN(s * g) and rD = RN(1 / D) are computed once per block.
+// Fast path: q = RN(|x| * rD) is within 2 ulp of the exact quotient, so the
+// hardware RNE of q decides the code unless q lies within a few ulp of a number
+// whose binary32 fraction has only its top two bits set — every E2M1 midpoint is
+// such a number.  Groups holding such an element take the exact comparison path.
+struct BlockEncoder {
+  float D, rD;
+  bool tiny;  // D < 2^-100: use the double comparison path for the whole block
+
+  __device__ __forceinline__ BlockEncoder(float D_) : D(D_) {
+    rD = (D > 0.0f) ? 1.0f / D : 0.0f;
+    tiny = D < 7.8886090522101181e-31f;  // 2^-100
+  }
+
+  __device__ __forceinline__ uint32_t index_slow(float ax) const {
+    return tiny ? e2m1_index_exact_f64(ax, D) : e2m1_index_exact(ax, D);
+  }
+
+  // 8 magnitudes -> 8 E2M1 indices packed into 32 bits (element k in bits 4k..4k+3)
+  __device__ __forceinline__ uint32_t encode8(const float (&ax)[8]) const {
+    if (!(D > 0.0f)) return 0u;
+    uint32_t word = 0;
+    bool any_slow = tiny;
+    float q[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      q[k] = ax[k] * rD;
+      const uint32_t u = __float_as_uint(q[k]);
+      const bool near = (((u + 4u) & 0x1FFFFFu) <= 8u) && q[k] > 0.125f && q[k] < 5.5f;
+      any_slow |= near;
+    }
+#pragma unroll
+    for (int k = 0; k < 8; k += 2) word |= e2m1x2_rn(q[k], q[k + 1]) << (4 * k);
+    if (any_slow) {
+      word = 0;
+#pragma unroll
+      for (int k = 0; k < 8; ++k) word |= index_slow(ax[k]) << (4 * k);
+    }
+    return word;
+  }
+};
+
+// Per-block scale: s = E4M3_RNE_sat(RN(amax_b / d6)) with d6 = RN(6 g); d6 == 0 -> 0.
+__device__ __forceinline__ uint32_t block_scale(float amax_b, float d6) {
+  if (!(d6 > 0.0f)) return 0u;
+  return e4m3_from_float(amax_b / d6);
+}
+
+// Sign bits of 8 floats -> bit 3 of each nibble (so -0 encodes as 0x8).
+__device__ __forceinline__ uint32_t f32_signs8(const float (&v)[8]) {
+  uint32_t r = 0;
+#pragma unroll
+  for (int k = 0; k < 8; ++k) r |= (__float_as_uint(v[k]) >> 31) << (4 * k + 3);
+  return r;
+}
+
+// Value of a 4-bit E2M1 code.
+__device__ __forceinline__ float e2m1_to_float(uint32_t c) {
+  // twice the magnitudes {0,0.5,1,1.5,2,3,4,6} = {0,1,2,3,4,6,8,12}, one nibble each
+  const float mag = __int2float_rn((int)((0xC8643210u >> (4 * (c & 7u))) & 0xFu)) * 0.5f;
+  return (c & 8u) ? -mag : mag;
+}
+
+// Offset of block scale (r, j) in the tensor-core (MMA) scale layout.
+__device__ __forceinline__ int64_t sf_mma_offset(int64_t r, int64_t j, int64_t groups) {
+  return ((r >> 7) * groups + (j >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (j & 3);
+}
+
+// Float <-> order-preserving signed int (for atomicMin/atomicMax on floats).
+__device__ __forceinline__ int float_to_ordered(float f) {
+  const int i = __float_as_int(f);
+  return i >= 0 ? i : i ^ 0x7FFFFFFF;
+}
+__device__ __forceinline__ float ordered_to_float(int i) {
+  return __int_as_float(i >= 0 ? i : i ^ 0x7FFFFFFF);
+}
+
+// Warp reductions
+__device__ __forceinline__ unsigned warp_max_u32(unsigned v) { return __reduce_max_sync(0xFFFFFFFFu, v); }
+
+// Fast unsigned division of 32-bit values by a runtime constant d >= 1
+// (round-up multiplier method, Granlund & Montgomery 1994):
+//   l = ceil(log2 d), m = floor(2^32 (2^l - d) / d) + 1,
+//   n / d = (t + ((n - t) >> 1)) >> (l - 1) with t = umulhi(n, m)   (d > 1).
+struct FastDiv {
+  uint32_t d, m, l;
+  __host__ FastDiv() : d(1), m(1), l(0) {}
+  __host__ explicit FastDiv(uint32_t d_) : d(d_), m(1), l(0) {
+    while ((1ull << l) < d) ++l;
+    m = (uint32_t)((((1ull << 32) * ((1ull << l) - d)) / d) + 1);
+  }
+  __device__ __forceinline__ uint32_t div(uint32_t n) const {
+    if (d == 1) return n;
+    const uint32_t t = __umulhi(n, m);
+    return (t + ((n - t) >> 1)) >> (l - 1);
+  }
+};
+
+}  // namespace nvfp4

@@ -1,0 +1,588 @@
+// gemm.cu — W4A4 block-scaled GEMM on the sm_100a tensor cores.
+//
+// techwalker.com, "NVIDIA研究团队打造全球首个FP4视频生成系统，速度提升两倍还省一半内存", §四:
+// all matmuls of the model run with 4-bit weights and activations; they are the
+// dominant cost of generation.  ai-manual.ru, "LongLive-2.0 ...", section
+// "Как это работает под капотом": scaling and quantization are merged into one
+// kernel — here the NVFP4 requantization of the activated output runs in the GEMM
+// epilogue.
+//
+//   c[m, n] = RN(acc[m, n] * RN(gA * gW)),   C = act(c)  (act: none or GELU-tanh)
+//   acc     = sum_k (e2m1(A[m,k]) sA[m,k/16]) (e2m1(W[n,k]) sW[n,k/16])  (FP32, tensor core)
+//
+// Structure: one persistent CTA per SM, 6 warps.
+//   warp 0      TMA producer: A and W code tiles (128 B swizzle, 128 rows x 256
+//               values per stage) and the stage's scale atoms (bulk copies).
+//   warp 1      MMA issuer: tcgen05.cp moves the scale atoms to tensor memory,
+//               tcgen05.mma.kind::mxf4nvf4.block_scale (UE4M3, 16-value blocks,
+//               K = 64 per instruction) accumulates into tensor memory.
+//   warps 2..5  epilogue: tcgen05.ld of the accumulator (one row per thread),
+//               scaling, optional GELU and NVFP4 requantization, stores.
+// Two accumulator buffers in tensor memory let the epilogue of one tile overlap
+// the main loop of the next.  No TMA load uses cluster multicast.
+//
+// Every wait is bounded: after ~2 s a wait records NVFP4_ERR_TIMEOUT in the
+// status word, raises a CTA-wide abort flag and the CTA drains its own
+// asynchronous work (bounded again) before it frees tensor memory and exits.
+#include <cuda.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int kBM = 128;           // tile rows (A rows, TMEM lanes)
+constexpr int kBN = 128;           // tile columns (W rows)
+constexpr int kBKBytes = 128;      // per stage: 128 bytes of packed codes = 256 values
+constexpr int kKPerMma = 64;       // values per tcgen05.mma (32 bytes)
+constexpr int kStages = 4;
+constexpr int kAccStages = 2;
+constexpr int kThreads = 192;
+constexpr int kEpiWarp0 = 2;
+constexpr int kTmemCols = 512;
+constexpr int kSfColBase = kAccStages * kBN;  // scale-factor columns follow the accumulators
+
+constexpr int kABytes = kBM * kBKBytes;        // 16 KB
+constexpr int kBBytes = kBN * kBKBytes;        // 16 KB
+constexpr int kSfaBytes = (kBM / 128) * 4 * 512;  // 4 atoms (one per 64-value group)
+constexpr int kSfbBytes = (kBN / 128) * 4 * 512;
+constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
+
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+struct Params {
+  int64_t M, N, K;
+  int64_t num_m, num_n, num_k64;  // tiles along M, N and 64-value groups along K
+  int64_t num_tiles;
+  int64_t sfa_row_tile_bytes;     // bytes of scale atoms per 128-row tile of A
+  int64_t sfw_row_tile_bytes;
+  const uint8_t* sfa;
+  const uint8_t* sfw;
+  const float* ga;
+  const float* gw;
+  uint8_t* c;
+  bool c_bf16;
+  int64_t ldc;
+  int act;
+  uint8_t* q_codes;
+  int64_t q_ld_codes;
+  uint8_t* q_scales;
+  int64_t q_groups;
+  const float* q_gscale_in;
+  float* q_gscale_out;
+  float* q_amax_out;
+  float* h_out;
+  unsigned* status;
+  unsigned long long wait_limit_ns;
+};
+
+// ----------------------------------------------------------------- PTX helpers
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
+               : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
+               "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the phase with `parity` to complete.  Returns false when the
+// wait gave up (time limit, or another role raised the abort flag).
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
+                                          unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > limit_ns) return false;
+    }
+  }
+}
+
+// Bounded wait that ignores the abort flag: used to drain this CTA's own
+// asynchronous copies and MMAs before it releases shared and tensor memory.
+__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const unsigned long long t0 = global_ns();
+  for (uint32_t it = 1;; ++it) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if ((it & 63u) == 0 && global_ns() - t0 > limit_ns) return false;
+  }
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
+                                            int32_t x, int32_t y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+      "l"(src), "r"(bytes), "r"(bar)
+      : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// Shared-memory matrix descriptor (tcgen05 format): start address, leading and
+// stride byte offsets (>> 4), descriptor version 1 at bits 46..47, layout type
+// at bits 61..63 (2 = 128-byte swizzle, 0 = no swizzle).
+__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
+  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
+  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
+  d |= (uint64_t)1 << 46;
+  d |= (uint64_t)(layout & 7u) << 61;
+  return d;
+}
+
+// Instruction descriptor of kind::mxf4nvf4 with UE4M3 scales: A and B E2M1
+// (format 1 at bits 7..9 and 10..12), both K-major, N >> 3 at bits 17..22,
+// scale format 0 (UE4M3) at bit 23, M >> 4 at bits 24..28, dense K = 64.
+constexpr uint32_t kIdesc = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) |
+                            ((uint32_t)(kBM >> 4) << 24);
+
+__device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
+                                             uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// 32 lanes x 128 bits from shared memory, replicated into the four 32-lane
+// quarters of tensor memory: the layout the block-scaled MMA reads its scales from.
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint32_t bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
+               : "memory");
+}
+
+// 32 consecutive 32-bit columns of this thread's lane.
+__device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]),
+        "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]),
+        "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ float gelu_tanh(float c) {
+  // 0.5 c (1 + tanh(sqrt(2/pi) (c + 0.044715 c^3)))
+  const float u = 0.7978845608028654f * (c + 0.044715f * (c * c * c));
+  return 0.5f * c * (1.0f + tanhf(u));
+}
+
+// ----------------------------------------------------------------- the kernel
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w,
+                Params p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* bar_area = smem + kStages * kStageBytes;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);
+  uint64_t* empty_bar = full_bar + kStages;
+  uint64_t* tfull_bar = empty_bar + kStages;
+  uint64_t* tempty_bar = tfull_bar + kAccStages;
+  uint64_t* done_bar = tempty_bar + kAccStages;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+    }
+    for (int a = 0; a < kAccStages; ++a) {
+      mbar_init(smem_u32(&tfull_bar[a]), 1);
+      mbar_init(smem_u32(&tempty_bar[a]), 4 * 32);
+    }
+    mbar_init(smem_u32(done_bar), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const unsigned long long limit = p.wait_limit_ns;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+      const int64_t kstages = (p.num_k64 + 3) / 4;
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+        const int64_t mt = tile % p.num_m, nt = tile / p.num_m;
+        for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1u;
+          if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag, limit)) {
+            ok = false;
+            break;
+          }
+          const int64_t g0 = ks * 4;
+          const int nvalid = (int)min((int64_t)4, p.num_k64 - g0);
+          uint8_t* st = smem + s * kStageBytes;
+          const uint32_t fb = smem_u32(&full_bar[s]);
+          mbar_arrive_expect_tx(fb, kABytes + kBBytes + 2 * nvalid * 512);
+          tma_load_2d(smem_u32(st), &map_a, fb, (int32_t)(ks * kBKBytes), (int32_t)(mt * kBM));
+          tma_load_2d(smem_u32(st + kABytes), &map_w, fb, (int32_t)(ks * kBKBytes), (int32_t)(nt * kBN));
+          bulk_load(smem_u32(st + kABytes + kBBytes), p.sfa + mt * p.sfa_row_tile_bytes + g0 * 512,
+                    nvalid * 512, fb);
+          bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes),
+                    p.sfw + nt * p.sfw_row_tile_bytes + g0 * 512, nvalid * 512, fb);
+        }
+      }
+      if (!ok) {
+        set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+      // drain: every load this thread issued must land before the CTA exits
+      const uint32_t n_issued = it;
+      for (uint32_t j = (n_issued > (uint32_t)kStages ? n_issued - kStages : 0); j < n_issued; ++j) {
+        const int s = j % kStages;
+        mbar_wait_drain(smem_u32(&full_bar[s]), (j / kStages) & 1u, limit);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const int64_t kstages = (p.num_k64 + 3) / 4;
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int64_t tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x, ++tcount) {
+        const int a = tcount % kAccStages;
+        const uint32_t aph = (tcount / kAccStages) & 1u;
+        if (!mbar_wait(smem_u32(&tempty_bar[a]), aph ^ 1u, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + a * kBN;
+        for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1u;
+          if (!mbar_wait(smem_u32(&full_bar[s]), ph, abort_flag, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nvalid = (int)min((int64_t)4, p.num_k64 - ks * 4);
+          uint8_t* st = smem + s * kStageBytes;
+          const uint32_t a_addr = smem_u32(st), b_addr = smem_u32(st + kABytes);
+          const uint32_t sfa_addr = smem_u32(st + kABytes + kBBytes);
+          const uint32_t sfb_addr = sfa_addr + kSfaBytes;
+          for (int k = 0; k < nvalid; ++k) {
+            const uint32_t sf_col = tmem_base + kSfColBase + (s * 4 + k) * 8;
+            tmem_cp_32x128b_warpx4(sf_col, smem_desc(sfa_addr + k * 512, 0, 128, 0));
+            tmem_cp_32x128b_warpx4(sf_col + 4, smem_desc(sfb_addr + k * 512, 0, 128, 0));
+            const uint64_t adesc = smem_desc(a_addr + k * 32, 16, 1024, 2);
+            const uint64_t bdesc = smem_desc(b_addr + k * 32, 16, 1024, 2);
+            mma_mxf4nvf4(d_tmem, adesc, bdesc, sf_col, sf_col + 4, (ks > 0 || k > 0) ? 1u : 0u);
+          }
+          mma_commit(smem_u32(&empty_bar[s]));
+        }
+        if (!ok) break;
+        mma_commit(smem_u32(&tfull_bar[a]));
+      }
+      if (!ok) {
+        set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+      // drain: all MMAs this thread issued complete before tensor memory is freed
+      mma_commit(smem_u32(done_bar));
+      mbar_wait_drain(smem_u32(done_bar), 0, limit);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // tensor-memory lanes this warp may access
+    const int row_in_tile = quarter * 32 + lane;
+    const float gab = (*p.ga) * (*p.gw);
+    float gq = 0.0f, d6q = 0.0f;
+    if (p.q_codes) {
+      gq = *p.q_gscale_in;
+      d6q = 6.0f * gq;
+      if (blockIdx.x == 0 && threadIdx.x == kEpiWarp0 * 32) *p.q_gscale_out = gq;
+    }
+    unsigned amax_bits = 0;
+    uint32_t tcount = 0;
+    for (int64_t tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
+      const int a = tcount % kAccStages;
+      const uint32_t aph = (tcount / kAccStages) & 1u;
+      // warp-uniform outcome: the tensor-memory loads below are warp-collective
+      const bool got = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&tfull_bar[a]), aph, abort_flag, limit));
+      if (!got) {
+        set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const int64_t mt = tile % p.num_m, nt = tile / p.num_m;
+      const int64_t row = mt * kBM + row_in_tile;
+      const bool row_ok = row < p.M;
+      for (int cc = 0; cc < kBN; cc += 32) {
+        uint32_t r[32];
+        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + a * kBN + cc;
+        tmem_ld_32x32b_x32(taddr, r);
+        const int64_t col0 = nt * kBN + cc;
+        if (!row_ok || col0 >= p.N) {
+          if (p.q_codes && !row_ok && col0 < p.N) {
+            // zero the scale padding of rows beyond M so the next GEMM reads finite scales
+            const int64_t j = col0 / 16;
+            if (row < (p.M + 127) / 128 * 128)
+              *reinterpret_cast<uint16_t*>(p.q_scales + sf_mma_offset(row, j, p.q_groups)) = 0;
+          }
+          continue;
+        }
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * gab;
+        if (col0 + 32 > p.N) {  // ragged last chunk (N % 32 == 16); never with q_codes
+          const int nv = (int)(p.N - col0);
+          for (int i = 0; i < nv; ++i) {
+            const float hv = p.act == 1 ? gelu_tanh(v[i]) : v[i];
+            if (p.c) {
+              if (p.c_bf16)
+                reinterpret_cast<uint16_t*>(p.c)[row * p.ldc + col0 + i] =
+                    (uint16_t)(pack_bf16x2(hv, 0.0f) & 0xFFFFu);
+              else
+                reinterpret_cast<float*>(p.c)[row * p.ldc + col0 + i] = hv;
+            }
+            if (p.h_out) p.h_out[row * p.N + col0 + i] = hv;
+            if (p.q_amax_out) amax_bits = max(amax_bits, __float_as_uint(hv) & 0x7FFFFFFFu);
+          }
+          continue;
+        }
+        if (p.act == 1) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
+        }
+        if (p.c) {
+          uint8_t* dst = p.c + (row * p.ldc + col0) * (p.c_bf16 ? 2 : 4);
+          if (p.c_bf16) {
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+              stg_v4(dst + 16 * q, make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]),
+                                              pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
+                                              pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
+                                              pack_bf16x2(v[8 * q + 6], v[8 * q + 7])));
+          } else {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              stg_v4(dst + 16 * q, make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                              __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3])));
+          }
+        }
+        if (p.h_out) {
+          float* hd = p.h_out + row * p.N + col0;
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            stg_v4(hd + 4 * q, make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                          __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3])));
+        }
+        if (p.q_amax_out) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) amax_bits = max(amax_bits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+        }
+        if (p.q_codes) {
+          uint32_t w[4];
+          uint32_t sc[2];
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            float ax[2][8], s0[8], s1[8];
+            float amax_b = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+              ax[k / 8][k % 8] = fabsf(v[16 * b + k]);
+              amax_b = fmaxf(amax_b, ax[k / 8][k % 8]);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              s0[k] = v[16 * b + k];
+              s1[k] = v[16 * b + 8 + k];
+            }
+            const uint32_t s = block_scale(amax_b, d6q);
+            const BlockEncoder enc(e4m3_to_float(s) * gq);
+            w[2 * b] = enc.encode8(ax[0]) | f32_signs8(s0);
+            w[2 * b + 1] = enc.encode8(ax[1]) | f32_signs8(s1);
+            sc[b] = s;
+          }
+          stg_v4(p.q_codes + row * p.q_ld_codes + col0 / 2, make_uint4(w[0], w[1], w[2], w[3]));
+          *reinterpret_cast<uint16_t*>(p.q_scales + sf_mma_offset(row, col0 / 16, p.q_groups)) =
+              (uint16_t)(sc[0] | (sc[1] << 8));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(smem_u32(&tempty_bar[a]));
+    }
+    if (p.q_amax_out) {
+      amax_bits = warp_max_u32(amax_bits);
+      if (lane == 0 && amax_bits) atomicMax(reinterpret_cast<unsigned*>(p.q_amax_out), amax_bits);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ----------------------------------------------------------------- host side
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+// 2-D map over packed codes: inner dimension K/2 bytes, outer `rows`; box of
+// 128 bytes x box_rows with the 128-byte swizzle the MMA descriptors assume.
+bool make_code_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t kbytes, int64_t ld,
+                   uint32_t box_rows) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)kbytes, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)ld};
+  cuuint32_t box[2] = {(cuuint32_t)kBKBytes, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
+  if (g.M == 0 || g.N == 0) return cudaSuccess;
+  Params p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.num_m = (g.M + kBM - 1) / kBM;
+  p.num_n = (g.N + kBN - 1) / kBN;
+  p.num_k64 = (g.K + kKPerMma - 1) / kKPerMma;
+  p.num_tiles = p.num_m * p.num_n;
+  p.sfa_row_tile_bytes = p.num_k64 * 512;
+  p.sfw_row_tile_bytes = p.num_k64 * 512;
+  p.sfa = g.a.scales;
+  p.sfw = g.w.scales;
+  p.ga = g.a.gscale;
+  p.gw = g.w.gscale;
+  p.c = (uint8_t*)g.c;
+  p.c_bf16 = g.c_bf16;
+  p.ldc = g.ldc;
+  p.act = g.act;
+  p.q_codes = g.q_codes;
+  p.q_ld_codes = g.q_ld_codes;
+  p.q_scales = g.q_scales;
+  p.q_groups = (g.N / 16 + 3) / 4;
+  p.q_gscale_in = g.q_gscale_in;
+  p.q_gscale_out = g.q_gscale_out;
+  p.q_amax_out = g.q_amax_out;
+  p.h_out = g.h_out;
+  p.status = g.status;
+  p.wait_limit_ns = kWaitLimitNs;
+
+  CUtensorMap ma, mw;
+  if (!make_code_map(&ma, g.a.codes, g.M, g.K / 2, g.a.ld_codes, kBM)) return cudaErrorInvalidValue;
+  if (!make_code_map(&mw, g.w.codes, g.N, g.K / 2, g.w.ld_codes, kBN)) return cudaErrorInvalidValue;
+
+  if (g.q_amax_out) {
+    cudaError_t e = cudaMemsetAsync(g.q_amax_out, 0, sizeof(float), s);
+    if (e != cudaSuccess) return e;
+  }
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int grid = (int)(p.num_tiles < sms ? p.num_tiles : sms);
+  gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mw, p);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,548 @@
+// kv.cu — NVFP4 KV cache: quantize-on-append (in place) and multi-chunk window
+// dequantization.
+//
+// techwalker.com, "NVIDIA研究团队打造全球首个FP4视频生成系统，速度提升两倍还省一半内存", §四:
+// K gets a simple mean subtraction, then K and V are stored in NVFP4; a dedicated
+// parallel CUDA kernel dequantizes several cache chunks of one window at once.
+// github.zuobiaodaohang.com, "长视频生成的两堵物理墙", section "NVFP4：数据体积砍到 1/4":
+// the quantized KV cache is updated in place.
+//
+// Reading fixed here: mu[h, d] = RN_f32(exact sum over the chunk's tokens / T),
+// K' = RN(k - mu), one tensor scale per chunk for K' and one for V, blocks of 16
+// along head_dim.  The exact sum makes mu independent of summation order.
+//
+// Append = 3 kernels on one stream:
+//   kv_stats_kernel : per (token split, column) double partial sums, min, max,
+//                     smallest nonzero |k|; max|v| (one read of K and V)
+//   kv_mu_kernel    : per column: mu (exact; see below), max|K'| over the chunk
+//   kv_encode_kernel: K' and V -> codes and scales of the slot (second read)
+// The double partial sums are exact whenever a column's nonzero magnitudes span at
+// most 45 - ceil(log2 T) binades (every value is then a multiple of the smallest
+// value's last bit and no partial sum can exceed 53 bits); a column outside that
+// range is summed exactly with integer limbs by kv_mu_kernel itself.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int kStatsThreads = 256;   // 8 warps; each lane owns 8 consecutive columns
+constexpr int kStatsCols = 256;      // columns per CTA
+constexpr int kSplits = 64;          // token splits of the stats pass
+constexpr int kMuThreads = 256;
+constexpr int kEncThreads = 256;
+constexpr int kMaxWindow = 64;
+
+// scratch layout (byte offsets from the scratch base)
+struct Scratch {
+  double* sum;     // [kSplits][C]
+  int* kmax;       // [kSplits][C] ordered ints
+  int* kmin;       // [kSplits][C]
+  unsigned* amin;  // [kSplits][C] smallest nonzero |k| bits (0xFFFFFFFF: none)
+  unsigned* words; // [0] max|v| bits, [1] max|K'| bits, [2] nonfinite flag
+};
+
+__host__ __device__ inline int64_t align256(int64_t x) { return (x + 255) / 256 * 256; }
+
+__host__ __device__ inline Scratch scratch_at(uint8_t* base, int64_t C) {
+  Scratch s;
+  int64_t o = 0;
+  s.sum = reinterpret_cast<double*>(base + o);
+  o += align256((int64_t)kSplits * C * 8);
+  s.kmax = reinterpret_cast<int*>(base + o);
+  o += align256((int64_t)kSplits * C * 4);
+  s.kmin = reinterpret_cast<int*>(base + o);
+  o += align256((int64_t)kSplits * C * 4);
+  s.amin = reinterpret_cast<unsigned*>(base + o);
+  o += align256((int64_t)kSplits * C * 4);
+  s.words = reinterpret_cast<unsigned*>(base + o);
+  return s;
+}
+
+struct StatsParams {
+  const uint8_t* k;
+  const uint8_t* v;
+  int64_t T, C;
+  int64_t tokens_per_split;
+  Scratch sc;
+};
+
+__global__ void __launch_bounds__(kStatsThreads) kv_stats_kernel(StatsParams p) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t c0 = (int64_t)blockIdx.x * kStatsCols + lane * 8;
+  const bool active = c0 < p.C;
+  const int split = blockIdx.y;
+  const int64_t t_begin = (int64_t)split * p.tokens_per_split;
+  const int64_t t_end = min(p.T, t_begin + p.tokens_per_split);
+
+  double sum[8];
+  float kmax[8], kmin[8];
+  unsigned amin[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    sum[i] = 0.0;
+    kmax[i] = -3.402823466e38f;
+    kmin[i] = 3.402823466e38f;
+    amin[i] = 0xFFFFFFFFu;
+  }
+  unsigned kbad = 0, vmax = 0;
+  if (active) {
+    for (int64_t t = t_begin + warp; t < t_end; t += kStatsThreads / 32) {
+      const uint4 kw = ldg_nc_v4(p.k + (t * p.C + c0) * 2);
+      const uint4 vw = ldg_nc_v4(p.v + (t * p.C + c0) * 2);
+      const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t bits = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
+        const float f = __uint_as_float(bits << 16);
+        sum[i] += (double)f;
+        kmax[i] = fmaxf(kmax[i], f);
+        kmin[i] = fminf(kmin[i], f);
+        const unsigned a = (bits & 0x7FFFu) << 16;
+        kbad = max(kbad, a);
+        amin[i] = min(amin[i], a ? a : 0xFFFFFFFFu);
+      }
+      vmax = __vmaxu2(vmax, vw.x & 0x7FFF7FFFu);
+      vmax = __vmaxu2(vmax, vw.y & 0x7FFF7FFFu);
+      vmax = __vmaxu2(vmax, vw.z & 0x7FFF7FFFu);
+      vmax = __vmaxu2(vmax, vw.w & 0x7FFF7FFFu);
+    }
+  }
+  vmax = max(vmax >> 16, vmax & 0xFFFFu) << 16;
+
+  // cross-warp reduction in shared memory, warp-major
+  __shared__ double s_sum[8][kStatsCols];
+  __shared__ float s_max[8][kStatsCols];
+  __shared__ float s_min[8][kStatsCols];
+  __shared__ unsigned s_amin[8][kStatsCols];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    s_sum[warp][lane * 8 + i] = sum[i];
+    s_max[warp][lane * 8 + i] = kmax[i];
+    s_min[warp][lane * 8 + i] = kmin[i];
+    s_amin[warp][lane * 8 + i] = amin[i];
+  }
+  __syncthreads();
+  const int64_t col = (int64_t)blockIdx.x * kStatsCols + threadIdx.x;
+  if (col < p.C) {
+    double s = 0.0;
+    float mx = -3.402823466e38f, mn = 3.402823466e38f;
+    unsigned am = 0xFFFFFFFFu;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      s += s_sum[w][threadIdx.x];
+      mx = fmaxf(mx, s_max[w][threadIdx.x]);
+      mn = fminf(mn, s_min[w][threadIdx.x]);
+      am = min(am, s_amin[w][threadIdx.x]);
+    }
+    const int64_t o = (int64_t)split * p.C + col;
+    p.sc.sum[o] = s;
+    p.sc.kmax[o] = float_to_ordered(mx);
+    p.sc.kmin[o] = float_to_ordered(mn);
+    p.sc.amin[o] = am;
+  }
+  // max|v| and the non-finite flag
+  const unsigned vm = warp_max_u32(vmax);
+  const unsigned kb = warp_max_u32(kbad);
+  if (lane == 0) {
+    if (vm) atomicMax(&p.sc.words[0], vm);
+    if (vm >= 0x7F800000u || kb >= 0x7F800000u) atomicOr(&p.sc.words[2], 1u);
+  }
+}
+
+// ------------------------------------------------------------- exact fallback
+
+// Unsigned integer with 32-bit digits in uint64 slots (lazy carries).
+constexpr int kLimbs = 10;
+
+__device__ int limbs_bitlen(const unsigned long long* n) {
+  for (int i = kLimbs - 1; i >= 0; --i)
+    if (n[i]) return i * 32 + 32 - __clz((unsigned)n[i]);
+  return 0;
+}
+
+// bit b of n (0 outside)
+__device__ unsigned limbs_bit(const unsigned long long* n, int b) {
+  if (b < 0 || b >= 32 * kLimbs) return 0;
+  return (unsigned)(n[b >> 5] >> (b & 31)) & 1u;
+}
+
+// RN_f32(N * 2^-133 / T), N given by normalized limbs (digits < 2^32):
+// take the top 64 bits of N (sticky for the rest), one 64-bit division by T
+// (the integer part is the same as that of N / (T 2^sh)), then round.
+__device__ float round_limbs_over_T(const unsigned long long* n, unsigned T, bool negative) {
+  const int L = limbs_bitlen(n);
+  if (L == 0) return 0.0f;
+  const int sh = L - 64;  // N = top * 2^sh + low
+  unsigned long long top = 0;
+  for (int b = L - 1; b >= max(sh, 0); --b) top = (top << 1) | limbs_bit(n, b);
+  if (sh < 0) top <<= -sh;
+  bool sticky = false;
+  for (int b = sh - 1; b >= 0 && !sticky; --b) sticky = limbs_bit(n, b);
+  const unsigned long long q = top / T;
+  sticky |= (top % T) != 0;
+  const int lq = 64 - __clzll((long long)q);
+  const int E = (lq - 1) + sh - 133;  // exponent of the leading bit
+  const int lsb = max(E - 23, -149);
+  // bits of q below the kept LSB: q has >= 33 significant bits, so a normal result
+  // drops lq - 24 >= 9 of them; a subnormal one (E < -126 forces sh < 8 - lq)
+  // drops -16 - sh, between 9 and 47.
+  const int drop = lsb - (sh - 133);
+  unsigned long long mant = q >> drop;
+  const unsigned guard = (unsigned)(q >> (drop - 1)) & 1u;
+  sticky |= (q & ((1ull << (drop - 1)) - 1ull)) != 0;
+  if (guard && (sticky || (mant & 1ull))) ++mant;
+  const float f = (float)ldexp((double)mant, lsb);
+  return negative ? -f : f;
+}
+
+__device__ void limbs_normalize(unsigned long long* n) {
+  for (int i = 0; i < kLimbs - 1; ++i) {
+    n[i + 1] += n[i] >> 32;
+    n[i] &= 0xFFFFFFFFull;
+  }
+}
+
+// RN_f32(S / T) for an exactly known double S: one double division, then fix the
+// only case where rounding twice can differ from rounding once — the double
+// quotient q landing exactly halfway between two binary32 neighbours while S / T
+// itself is not halfway.
+__device__ float mean_from_exact_double(double S, unsigned T) {
+  const double q = S / (double)T;
+  const float f = (float)q;
+  const double fd = (double)f;
+  if (q != fd) {
+    const float nb = q > fd ? nextafterf(f, 3.402823466e38f) : nextafterf(f, -3.402823466e38f);
+    if (q == 0.5 * (fd + (double)nb)) {
+      const double r = fma(-q, (double)T, S);  // exact sign of S/T - q
+      if (r != 0.0) return r > 0.0 ? fmaxf(f, nb) : fminf(f, nb);
+    }
+  }
+  return f;
+}
+
+struct MuParams {
+  const uint8_t* k;
+  int64_t T, C;
+  Scratch sc;
+  float* mu;   // slot's mu [C]
+  int log2T_ceil;
+};
+
+__global__ void __launch_bounds__(kMuThreads) kv_mu_kernel(MuParams p) {
+  if (p.sc.words[2]) return;  // non-finite input: the slot stays unchanged
+  const int64_t c = (int64_t)blockIdx.x * kMuThreads + threadIdx.x;
+  double S = 0.0;
+  float kmax = -3.402823466e38f, kmin = 3.402823466e38f;
+  unsigned amin = 0xFFFFFFFFu;
+  bool exact = true;
+  if (c < p.C) {
+    for (int sp = 0; sp < kSplits; ++sp) {
+      const int64_t o = (int64_t)sp * p.C + c;
+      S += p.sc.sum[o];
+      kmax = fmaxf(kmax, ordered_to_float(p.sc.kmax[o]));
+      kmin = fminf(kmin, ordered_to_float(p.sc.kmin[o]));
+      amin = min(amin, p.sc.amin[o]);
+    }
+    if (amin != 0xFFFFFFFFu) {
+      const float amax = fmaxf(fabsf(kmax), fabsf(kmin));
+      const int e_max = max((int)((__float_as_uint(amax) >> 23) & 0xFF), 1);
+      const int e_min = max((int)((amin >> 23) & 0xFF), 1);
+      exact = (e_max - e_min) <= 45 - p.log2T_ceil;
+    }
+  }
+  __shared__ int n_inexact;
+  __shared__ int inexact_cols[kMuThreads];
+  __shared__ float inexact_mu[kMuThreads];
+  __shared__ unsigned long long limbs[2][kLimbs];
+  if (threadIdx.x == 0) n_inexact = 0;
+  __syncthreads();
+  if (c < p.C && !exact) inexact_cols[atomicAdd(&n_inexact, 1)] = threadIdx.x;
+  __syncthreads();
+  // exact integer-limb sums for the (rare) columns outside the double's range
+  for (int i = 0; i < n_inexact; ++i) {
+    const int64_t cc = (int64_t)blockIdx.x * kMuThreads + inexact_cols[i];
+    if (threadIdx.x < 2 * kLimbs) limbs[threadIdx.x / kLimbs][threadIdx.x % kLimbs] = 0;
+    __syncthreads();
+    for (int64_t t = threadIdx.x; t < p.T; t += kMuThreads) {
+      const unsigned b = *reinterpret_cast<const unsigned short*>(p.k + (t * p.C + cc) * 2);
+      const unsigned e = (b >> 7) & 0xFFu, m = b & 0x7Fu;
+      if (e == 0 && m == 0) continue;
+      const unsigned long long mant = e ? (128u + m) : m;  // value = mant * 2^(pos - 133)
+      const int pos = e ? (int)e - 1 : 0;
+      atomicAdd(&limbs[b >> 15][pos >> 5], mant << (pos & 31));
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      unsigned long long* P = limbs[0];
+      unsigned long long* N = limbs[1];
+      limbs_normalize(P);
+      limbs_normalize(N);
+      int cmp = 0;
+      for (int d = kLimbs - 1; d >= 0 && cmp == 0; --d)
+        cmp = P[d] > N[d] ? 1 : (P[d] < N[d] ? -1 : 0);
+      unsigned long long mag[kLimbs];
+      const unsigned long long* big = cmp >= 0 ? P : N;
+      const unsigned long long* small = cmp >= 0 ? N : P;
+      long long borrow = 0;
+      for (int d = 0; d < kLimbs; ++d) {
+        long long t = (long long)big[d] - (long long)small[d] - borrow;
+        borrow = t < 0;
+        mag[d] = (unsigned long long)(t + (borrow ? (1ll << 32) : 0));
+      }
+      inexact_mu[i] = cmp == 0 ? 0.0f : round_limbs_over_T(mag, (unsigned)p.T, cmp < 0);
+    }
+    __syncthreads();
+  }
+  if (c >= p.C) return;
+  float mu;
+  if (!exact) {
+    mu = 0.0f;
+    for (int i = 0; i < n_inexact; ++i)
+      if (inexact_cols[i] == (int)threadIdx.x) mu = inexact_mu[i];
+  } else {
+    mu = (amin == 0xFFFFFFFFu) ? 0.0f : mean_from_exact_double(S, (unsigned)p.T);
+  }
+  p.mu[c] = mu;
+  // max |RN(k - mu)| over the column is reached at its max or its min (RN is monotone)
+  const float a = fmaxf(fabsf(kmax - mu), fabsf(kmin - mu));
+  atomicMax(&p.sc.words[1], __float_as_uint(a));
+}
+
+struct EncParams {
+  const uint8_t* k;
+  const uint8_t* v;
+  int64_t nblocks;    // T * C / 16
+  FastDiv cblocks;    // C / 16
+  const float* mu;
+  uint8_t* k_codes;
+  uint8_t* v_codes;
+  uint8_t* k_scales;
+  uint8_t* v_scales;
+  float* gscale;      // slot's (g_K, g_V)
+  const unsigned* words;
+};
+
+__device__ __forceinline__ void encode_block16(const float (&v)[16], float g, float d6,
+                                               uint8_t* codes, uint8_t* scale) {
+  float ax[2][8], v0[8], v1[8];
+  float amax_b = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    ax[k / 8][k % 8] = fabsf(v[k]);
+    amax_b = fmaxf(amax_b, fabsf(v[k]));
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    v0[k] = v[k];
+    v1[k] = v[8 + k];
+  }
+  const uint32_t s = block_scale(amax_b, d6);
+  const BlockEncoder enc(e4m3_to_float(s) * g);
+  uint2 out;
+  out.x = enc.encode8(ax[0]) | f32_signs8(v0);
+  out.y = enc.encode8(ax[1]) | f32_signs8(v1);
+  stg_v2(codes, out);
+  *scale = (uint8_t)s;
+}
+
+__global__ void __launch_bounds__(kEncThreads) kv_encode_kernel(EncParams p) {
+  if (p.words[2]) return;
+  const float gk = __uint_as_float(p.words[1]) / 2688.0f;
+  const float gv = __uint_as_float(p.words[0]) / 2688.0f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    p.gscale[0] = gk;
+    p.gscale[1] = gv;
+  }
+  const float d6k = 6.0f * gk, d6v = 6.0f * gv;
+  const int64_t stride = (int64_t)gridDim.x * kEncThreads;
+  for (int64_t b = (int64_t)blockIdx.x * kEncThreads + threadIdx.x; b < p.nblocks; b += stride) {
+    const uint32_t row = p.cblocks.div((uint32_t)b);
+    const int64_t c = ((int64_t)b - (int64_t)row * p.cblocks.d) * 16;
+    float kv[16], vv[16];
+    {
+      const uint4 a = ldg_nc_v4(p.k + b * 32), bb = ldg_nc_v4(p.k + b * 32 + 16);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, bb.x, bb.y, bb.z, bb.w};
+      const float4* m4 = reinterpret_cast<const float4*>(p.mu + c);
+      float mu[16];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const float4 m = m4[q];
+        mu[4 * q] = m.x;
+        mu[4 * q + 1] = m.y;
+        mu[4 * q + 2] = m.z;
+        mu[4 * q + 3] = m.w;
+      }
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        kv[2 * q] = bf16_lo(w[q]) - mu[2 * q];
+        kv[2 * q + 1] = bf16_hi(w[q]) - mu[2 * q + 1];
+      }
+    }
+    {
+      const uint4 a = ldg_nc_v4(p.v + b * 32), bb = ldg_nc_v4(p.v + b * 32 + 16);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, bb.x, bb.y, bb.z, bb.w};
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        vv[2 * q] = bf16_lo(w[q]);
+        vv[2 * q + 1] = bf16_hi(w[q]);
+      }
+    }
+    encode_block16(kv, gk, d6k, p.k_codes + b * 8, p.k_scales + b);
+    encode_block16(vv, gv, d6v, p.v_codes + b * 8, p.v_scales + b);
+  }
+}
+
+struct WindowParams {
+  const uint8_t* base;
+  int64_t off_k_codes, off_v_codes, off_k_scales, off_v_scales, off_mu, off_gscale;
+  int64_t slot_codes_bytes, slot_scales_bytes, C;
+  int64_t blocks_per_chunk;  // T * C / 16
+  FastDiv bpc, cblocks;
+  int64_t nblocks;           // n_slots * blocks_per_chunk
+  int32_t slots[kMaxWindow];
+  uint8_t* k_out;
+  uint8_t* v_out;
+};
+
+// One thread produces one 16-value block of K^ and of V^.
+__global__ void __launch_bounds__(kEncThreads) kv_window_kernel(WindowParams p) {
+  const int64_t stride = (int64_t)gridDim.x * kEncThreads;
+  for (int64_t ob = (int64_t)blockIdx.x * kEncThreads + threadIdx.x; ob < p.nblocks; ob += stride) {
+    const uint32_t i = p.bpc.div((uint32_t)ob);
+    const int64_t b = ob - (int64_t)i * p.blocks_per_chunk;
+    const int64_t slot = p.slots[i];
+    const uint32_t row = p.cblocks.div((uint32_t)b);
+    const int64_t c = (b - (int64_t)row * p.cblocks.d) * 16;
+    const float* g = reinterpret_cast<const float*>(p.base + p.off_gscale) + 2 * slot;
+    const float gk = g[0], gv = g[1];
+    const uint2 kc = *reinterpret_cast<const uint2*>(p.base + p.off_k_codes + slot * p.slot_codes_bytes + b * 8);
+    const uint2 vc = *reinterpret_cast<const uint2*>(p.base + p.off_v_codes + slot * p.slot_codes_bytes + b * 8);
+    const float ks = e4m3_to_float(p.base[p.off_k_scales + slot * p.slot_scales_bytes + b]);
+    const float vs = e4m3_to_float(p.base[p.off_v_scales + slot * p.slot_scales_bytes + b]);
+    const float4* m4 = reinterpret_cast<const float4*>(p.base + p.off_mu + (slot * p.C + c) * 4);
+    float mu[16];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const float4 m = m4[q];
+      mu[4 * q] = m.x;
+      mu[4 * q + 1] = m.y;
+      mu[4 * q + 2] = m.z;
+      mu[4 * q + 3] = m.w;
+    }
+    float ko[16], vo[16];
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      const uint32_t kcode = ((q < 8 ? kc.x : kc.y) >> (4 * (q & 7))) & 0xFu;
+      const uint32_t vcode = ((q < 8 ? vc.x : vc.y) >> (4 * (q & 7))) & 0xFu;
+      ko[q] = (e2m1_to_float(kcode) * ks) * gk + mu[q];  // no fusion: -fmad=false
+      vo[q] = (e2m1_to_float(vcode) * vs) * gv;
+    }
+    uint8_t* kd = p.k_out + ob * 32;
+    uint8_t* vd = p.v_out + ob * 32;
+    stg_v4(kd, make_uint4(pack_bf16x2(ko[0], ko[1]), pack_bf16x2(ko[2], ko[3]),
+                          pack_bf16x2(ko[4], ko[5]), pack_bf16x2(ko[6], ko[7])));
+    stg_v4(kd + 16, make_uint4(pack_bf16x2(ko[8], ko[9]), pack_bf16x2(ko[10], ko[11]),
+                               pack_bf16x2(ko[12], ko[13]), pack_bf16x2(ko[14], ko[15])));
+    stg_v4(vd, make_uint4(pack_bf16x2(vo[0], vo[1]), pack_bf16x2(vo[2], vo[3]),
+                          pack_bf16x2(vo[4], vo[5]), pack_bf16x2(vo[6], vo[7])));
+    stg_v4(vd + 16, make_uint4(pack_bf16x2(vo[8], vo[9]), pack_bf16x2(vo[10], vo[11]),
+                               pack_bf16x2(vo[12], vo[13]), pack_bf16x2(vo[14], vo[15])));
+  }
+}
+
+int sm_count() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+}  // namespace
+
+int64_t kv_scratch_bytes(int32_t heads, int32_t head_dim, int64_t chunk_tokens) {
+  (void)chunk_tokens;
+  const int64_t C = (int64_t)heads * head_dim;
+  return align256((int64_t)kSplits * C * 8) + 3 * align256((int64_t)kSplits * C * 4) + 256;
+}
+
+cudaError_t launch_kv_append(const KVLayout& L, const void* k, const void* v, int32_t slot,
+                             unsigned* status, cudaStream_t s) {
+  (void)status;
+  const int64_t C = (int64_t)L.heads * L.head_dim;
+  const int64_t T = L.chunk_tokens;
+  Scratch sc = scratch_at(L.base + L.off_scratch, C);
+  cudaError_t e = cudaMemsetAsync(sc.words, 0, 3 * sizeof(unsigned), s);
+  if (e != cudaSuccess) return e;
+
+  StatsParams sp;
+  sp.k = (const uint8_t*)k;
+  sp.v = (const uint8_t*)v;
+  sp.T = T;
+  sp.C = C;
+  sp.tokens_per_split = (T + kSplits - 1) / kSplits;
+  sp.sc = sc;
+  dim3 sgrid((unsigned)((C + kStatsCols - 1) / kStatsCols), kSplits);
+  kv_stats_kernel<<<sgrid, kStatsThreads, 0, s>>>(sp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  MuParams mp;
+  mp.k = (const uint8_t*)k;
+  mp.T = T;
+  mp.C = C;
+  mp.sc = sc;
+  mp.mu = reinterpret_cast<float*>(L.base + L.off_mu) + (int64_t)slot * C;
+  int lg = 0;
+  while ((1ll << lg) < T) ++lg;
+  mp.log2T_ceil = lg;
+  kv_mu_kernel<<<(unsigned)((C + kMuThreads - 1) / kMuThreads), kMuThreads, 0, s>>>(mp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  EncParams ep;
+  ep.k = (const uint8_t*)k;
+  ep.v = (const uint8_t*)v;
+  ep.nblocks = T * C / 16;
+  ep.cblocks = FastDiv((uint32_t)(C / 16));
+  ep.mu = mp.mu;
+  ep.k_codes = L.base + L.off_k_codes + (int64_t)slot * L.slot_codes_bytes;
+  ep.v_codes = L.base + L.off_v_codes + (int64_t)slot * L.slot_codes_bytes;
+  ep.k_scales = L.base + L.off_k_scales + (int64_t)slot * L.slot_scales_bytes;
+  ep.v_scales = L.base + L.off_v_scales + (int64_t)slot * L.slot_scales_bytes;
+  ep.gscale = reinterpret_cast<float*>(L.base + L.off_gscale) + 2 * (int64_t)slot;
+  ep.words = sc.words;
+  const int64_t want = (ep.nblocks + kEncThreads - 1) / kEncThreads;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  kv_encode_kernel<<<(unsigned)(want < cap ? want : cap), kEncThreads, 0, s>>>(ep);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  // a non-finite input is reported through the sticky status word
+  return cudaSuccess;
+}
+
+cudaError_t launch_kv_window(const KVLayout& L, const int32_t* slots, int32_t n_slots, void* k_out,
+                             void* v_out, cudaStream_t s) {
+  WindowParams p;
+  p.base = L.base;
+  p.off_k_codes = L.off_k_codes;
+  p.off_v_codes = L.off_v_codes;
+  p.off_k_scales = L.off_k_scales;
+  p.off_v_scales = L.off_v_scales;
+  p.off_mu = L.off_mu;
+  p.off_gscale = L.off_gscale;
+  p.slot_codes_bytes = L.slot_codes_bytes;
+  p.slot_scales_bytes = L.slot_scales_bytes;
+  p.C = (int64_t)L.heads * L.head_dim;
+  p.blocks_per_chunk = L.chunk_tokens * p.C / 16;
+  p.bpc = FastDiv((uint32_t)p.blocks_per_chunk);
+  p.cblocks = FastDiv((uint32_t)(p.C / 16));
+  p.nblocks = (int64_t)n_slots * p.blocks_per_chunk;
+  for (int i = 0; i < kMaxWindow; ++i) p.slots[i] = i < n_slots ? slots[i] : 0;
+  p.k_out = (uint8_t*)k_out;
+  p.v_out = (uint8_t*)v_out;
+  const int64_t want = (p.nblocks + kEncThreads - 1) / kEncThreads;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  kv_window_kernel<<<(unsigned)(want < cap ? want : cap), kEncThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

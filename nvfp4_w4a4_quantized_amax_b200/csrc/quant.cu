@@ -1,0 +1,301 @@
+// quant.cu — NVFP4 activation quantization and dequantization (HBM-bound).
+//
+// techwalker.com, "NVIDIA研究团队打造全球首个FP4视频生成系统，速度提升两倍还省一半内存", §一:
+// every 16 values share one FP8 scale and the whole tensor shares one FP32 scale.
+// The tensor scale needs max|x| before any block can be encoded, so quantization
+// with an unknown scale is two passes over x: amax_kernel, then encode_kernel.
+// With a supplied scale (one pass) encode_kernel also reports max|x| for the
+// caller's next calibration.
+//
+// Memory traffic per element (bf16 in): amax pass 2 B read; encode pass 2 B read,
+// 0.5 B codes + 1/16 B scale written.  Loads are 128-bit and read-only-path.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ void block_max_atomic(unsigned v, unsigned* dst) {
+  __shared__ unsigned red[kThreads / 32];
+  v = warp_max_u32(v);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane == 0) red[warp] = v;
+  __syncthreads();
+  if (warp == 0) {
+    v = lane < kThreads / 32 ? red[lane] : 0u;
+    v = warp_max_u32(v);
+    if (lane == 0 && v != 0u) atomicMax(dst, v);
+  }
+}
+
+// max |x| as binary32 bits (non-negative floats order like unsigned integers; a
+// NaN or Inf anywhere yields bits >= 0x7F800000).  x is read in 16-byte chunks,
+// chunks_per_row per row.
+template <bool kBf16>
+__global__ void __launch_bounds__(kThreads) amax_kernel(const uint8_t* __restrict__ x,
+                                                        int64_t row_bytes, int64_t nchunks,
+                                                        FastDiv cpr, unsigned* amax_bits) {
+  unsigned m = 0;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nchunks; i += stride) {
+    const uint32_t r = cpr.div((uint32_t)i);
+    const uint32_t c = (uint32_t)i - r * cpr.d;
+    const uint4 v = ldg_nc_v4(x + (int64_t)r * row_bytes + (int64_t)c * 16);
+    if (kBf16) {
+      m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+    } else {
+      m = max(m, v.x & 0x7FFFFFFFu);
+      m = max(m, v.y & 0x7FFFFFFFu);
+      m = max(m, v.z & 0x7FFFFFFFu);
+      m = max(m, v.w & 0x7FFFFFFFu);
+    }
+  }
+  if (kBf16) m = max(m >> 16, m & 0xFFFFu) << 16;
+  block_max_atomic(m, amax_bits);
+}
+
+struct EncodeParams {
+  const uint8_t* x;
+  int64_t x_row_bytes;
+  uint8_t* codes;
+  int64_t ld_codes;
+  uint8_t* scales;
+  int64_t ld_scales;
+  int64_t groups;   // MMA layout: ceil(nb / 4)
+  int64_t rows, nb; // real rows and blocks per row
+  int64_t nvblocks; // blocks visited (includes MMA-layout padding)
+  FastDiv vb_per_row;
+  const float* gscale_in;
+  const unsigned* amax_bits;
+  float* gscale_out;
+  unsigned* amax_accum;  // nullable (one-pass mode)
+  unsigned* status;
+};
+
+// One thread encodes one 16-value block: block amax -> E4M3 scale -> 16 codes.
+template <bool kBf16, bool kMma>
+__global__ void __launch_bounds__(kThreads) encode_kernel(EncodeParams p) {
+  float g;
+  if (p.gscale_in) {
+    g = *p.gscale_in;
+    if (!(g >= 0.0f) || !(g <= 3.402823466e38f)) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) set_status(p.status, kStatusNonfinite);
+      return;
+    }
+  } else {
+    const unsigned ab = *p.amax_bits;
+    if (ab >= 0x7F800000u) {
+      if (blockIdx.x == 0 && threadIdx.x == 0) set_status(p.status, kStatusNonfinite);
+      return;
+    }
+    g = __uint_as_float(ab) / 2688.0f;
+  }
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.gscale_out = g;
+  const float d6 = 6.0f * g;
+
+  unsigned local_max = 0;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t vb = (int64_t)blockIdx.x * kThreads + threadIdx.x; vb < p.nvblocks; vb += stride) {
+    const uint32_t r = p.vb_per_row.div((uint32_t)vb);
+    const uint32_t j = (uint32_t)vb - r * p.vb_per_row.d;
+    const int64_t soff = kMma ? sf_mma_offset(r, j, p.groups) : (int64_t)r * p.ld_scales + j;
+    if (kMma && (r >= p.rows || j >= p.nb)) {  // padding of the tensor-core layout
+      p.scales[soff] = 0;
+      continue;
+    }
+    float v[16];
+    const uint8_t* src = p.x + (int64_t)r * p.x_row_bytes + (int64_t)j * (kBf16 ? 32 : 64);
+    if (kBf16) {
+      const uint4 a = ldg_nc_v4(src), b = ldg_nc_v4(src + 16);
+      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        v[2 * k] = bf16_lo(w[k]);
+        v[2 * k + 1] = bf16_hi(w[k]);
+      }
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const uint4 a = ldg_nc_v4(src + 16 * k);
+        v[4 * k] = __uint_as_float(a.x);
+        v[4 * k + 1] = __uint_as_float(a.y);
+        v[4 * k + 2] = __uint_as_float(a.z);
+        v[4 * k + 3] = __uint_as_float(a.w);
+      }
+    }
+    float amax_b = 0.0f;
+    float ax[2][8];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      ax[k / 8][k % 8] = fabsf(v[k]);
+      amax_b = fmaxf(amax_b, ax[k / 8][k % 8]);
+    }
+    if (p.amax_accum) {
+      unsigned bits = 0;
+#pragma unroll
+      for (int k = 0; k < 16; ++k) bits = max(bits, __float_as_uint(v[k]) & 0x7FFFFFFFu);
+      local_max = max(local_max, bits);
+    }
+    const uint32_t s = block_scale(amax_b, d6);
+    const BlockEncoder enc(e4m3_to_float(s) * g);
+    float v0[8], v1[8];
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      v0[k] = v[k];
+      v1[k] = v[8 + k];
+    }
+    uint2 out;
+    out.x = enc.encode8(ax[0]) | f32_signs8(v0);
+    out.y = enc.encode8(ax[1]) | f32_signs8(v1);
+    stg_v2(p.codes + (int64_t)r * p.ld_codes + (int64_t)j * 8, out);
+    p.scales[soff] = (uint8_t)s;
+  }
+  if (p.amax_accum) {
+    if (local_max >= 0x7F800000u) set_status(p.status, kStatusNonfinite);
+    block_max_atomic(local_max, p.amax_accum);
+  }
+}
+
+struct DequantParams {
+  const uint8_t* codes;
+  int64_t ld_codes;
+  const uint8_t* scales;
+  int64_t ld_scales;
+  int64_t groups;
+  const float* gscale;
+  int64_t nblocks;
+  FastDiv nb_per_row;
+  uint8_t* y;
+  int64_t y_row_bytes;
+};
+
+// One thread decodes one 16-value block: y = RN(RN(e2m1 * s) * g).
+template <bool kMma, bool kBf16Out>
+__global__ void __launch_bounds__(kThreads) dequant_kernel(DequantParams p) {
+  const float g = *p.gscale;
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < p.nblocks; b += stride) {
+    const uint32_t r = p.nb_per_row.div((uint32_t)b);
+    const uint32_t j = (uint32_t)b - r * p.nb_per_row.d;
+    const uint2 c = *reinterpret_cast<const uint2*>(p.codes + (int64_t)r * p.ld_codes + (int64_t)j * 8);
+    const int64_t soff = kMma ? sf_mma_offset(r, j, p.groups) : (int64_t)r * p.ld_scales + j;
+    const float s = e4m3_to_float(p.scales[soff]);
+    float y[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      const uint32_t code = ((k < 8 ? c.x : c.y) >> (4 * (k & 7))) & 0xFu;
+      y[k] = (e2m1_to_float(code) * s) * g;  // the first product is exact
+    }
+    uint8_t* dst = p.y + (int64_t)r * p.y_row_bytes + (int64_t)j * (kBf16Out ? 32 : 64);
+    if (kBf16Out) {
+      stg_v4(dst, make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
+                             pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7])));
+      stg_v4(dst + 16, make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]),
+                                  pack_bf16x2(y[12], y[13]), pack_bf16x2(y[14], y[15])));
+    } else {
+#pragma unroll
+      for (int k = 0; k < 4; ++k)
+        stg_v4(dst + 16 * k, make_uint4(__float_as_uint(y[4 * k]), __float_as_uint(y[4 * k + 1]),
+                                        __float_as_uint(y[4 * k + 2]), __float_as_uint(y[4 * k + 3])));
+    }
+  }
+}
+
+int grid_for(int64_t work) {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  const int64_t want = (work + kThreads - 1) / kThreads;
+  const int64_t cap = (int64_t)sms * 8;
+  return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
+}  // namespace
+
+cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
+  const int64_t esz = a.x_bf16 ? 2 : 4;
+  const int64_t nb = a.cols / 16;
+  unsigned* amax_bits = reinterpret_cast<unsigned*>(a.amax_out);
+  if (a.amax_out) {
+    cudaError_t e = cudaMemsetAsync(a.amax_out, 0, sizeof(float), s);
+    if (e != cudaSuccess) return e;
+  }
+  if (a.rows == 0) {
+    if (!a.gscale_in) {  // empty tensor: amax = 0, g = 0
+      return cudaMemsetAsync(a.gscale_out, 0, sizeof(float), s);
+    }
+    return cudaMemcpyAsync(a.gscale_out, a.gscale_in, sizeof(float), cudaMemcpyDeviceToDevice, s);
+  }
+  if (!a.gscale_in) {
+    const int64_t cpr = a.cols * esz / 16;
+    const int64_t n = a.rows * cpr;
+    if (a.x_bf16)
+      amax_kernel<true><<<grid_for(n), kThreads, 0, s>>>((const uint8_t*)a.x, a.ldx * esz, n,
+                                                         FastDiv((uint32_t)cpr), amax_bits);
+    else
+      amax_kernel<false><<<grid_for(n), kThreads, 0, s>>>((const uint8_t*)a.x, a.ldx * esz, n,
+                                                          FastDiv((uint32_t)cpr), amax_bits);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  EncodeParams p;
+  p.x = (const uint8_t*)a.x;
+  p.x_row_bytes = a.ldx * esz;
+  p.codes = a.codes;
+  p.ld_codes = a.ld_codes;
+  p.scales = a.scales;
+  p.ld_scales = a.ld_scales;
+  p.groups = (nb + 3) / 4;
+  p.rows = a.rows;
+  p.nb = nb;
+  const int64_t vb_per_row = a.sf_mma ? p.groups * 4 : nb;
+  const int64_t vrows = a.sf_mma ? (a.rows + 127) / 128 * 128 : a.rows;
+  p.nvblocks = vrows * vb_per_row;
+  p.vb_per_row = FastDiv((uint32_t)vb_per_row);
+  p.gscale_in = a.gscale_in;
+  p.amax_bits = amax_bits;
+  p.gscale_out = a.gscale_out;
+  p.amax_accum = a.gscale_in ? amax_bits : nullptr;
+  p.status = a.status;
+  const int grid = grid_for(p.nvblocks);
+  if (a.x_bf16) {
+    if (a.sf_mma) encode_kernel<true, true><<<grid, kThreads, 0, s>>>(p);
+    else encode_kernel<true, false><<<grid, kThreads, 0, s>>>(p);
+  } else {
+    if (a.sf_mma) encode_kernel<false, true><<<grid, kThreads, 0, s>>>(p);
+    else encode_kernel<false, false><<<grid, kThreads, 0, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t s) {
+  if (a.rows == 0) return cudaSuccess;
+  DequantParams p;
+  p.codes = a.codes;
+  p.ld_codes = a.ld_codes;
+  p.scales = a.scales;
+  p.ld_scales = a.ld_scales;
+  const int64_t nb = a.cols / 16;
+  p.groups = (nb + 3) / 4;
+  p.gscale = a.gscale;
+  p.nblocks = a.rows * nb;
+  p.nb_per_row = FastDiv((uint32_t)nb);
+  p.y = (uint8_t*)a.y;
+  p.y_row_bytes = a.ldy * (a.y_bf16 ? 2 : 4);
+  const int grid = grid_for(p.nblocks);
+  if (a.sf_mma) {
+    if (a.y_bf16) dequant_kernel<true, true><<<grid, kThreads, 0, s>>>(p);
+    else dequant_kernel<true, false><<<grid, kThreads, 0, s>>>(p);
+  } else {
+    if (a.y_bf16) dequant_kernel<false, true><<<grid, kThreads, 0, s>>>(p);
+    else dequant_kernel<false, false><<<grid, kThreads, 0, s>>>(p);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

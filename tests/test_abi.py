@@ -1,0 +1,112 @@
+"""The C-ABI library: it loads, exports every entry point that include/nvfp4.h
+declares, and rejects bad arguments on the host before touching a device.  CPU only
+(no call here reaches a kernel)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import nvfp4_w4a4_quantized_amax_b200 as nv
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "nvfp4.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\**\s+([A-Za-z_][A-Za-z0-9_]*)\s*\(",
+                       text, flags=re.M)
+    return sorted(set(n for n in names if n not in ("if", "return")))
+
+
+def test_header_declares_the_hot_path_calls():
+    names = declared_functions()
+    for n in ["nvfp4_quantize", "nvfp4_dequantize", "nvfp4_gemm", "kv_quant_append",
+              "kv_dequant_window"]:
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol():
+    lib = nv.library()
+    missing = [n for n in declared_functions() if not hasattr(lib, n)]
+    assert not missing, missing
+    assert sorted(declared_functions()) == sorted(nv.EXPORTS)
+
+
+def test_version_and_status_strings():
+    lib = nv.library()
+    assert lib.nvfp4_version() >> 16 == 1
+    assert nv.status_string(nv.OK) == "ok"
+    assert "non-finite" in nv.status_string(nv.ERR_NONFINITE)
+
+
+def test_scale_sizes():
+    assert nv.scales_bytes(128, 512, nv.SF_ROWMAJOR) == 128 * 32
+    assert nv.scales_bytes(130, 48, nv.SF_MMA) == 256 * 4
+    assert nv.scales_bytes(8192, 3072, nv.SF_MMA) == 8192 * 192
+    with pytest.raises(nv.Nvfp4Error) as e:
+        nv.scales_bytes(4, 24, nv.SF_MMA)
+    assert e.value.status == nv.ERR_SHAPE
+
+
+def test_kv_cache_geometry_matches_storage_claim():
+    heads, dh, T, chunks = 24, 128, 8192, 16
+    nbytes = nv.kv_cache_bytes(heads, dh, T, chunks)
+    pairs = heads * dh * T * chunks
+    codes_and_scales = 2 * (pairs // 2 + pairs // 16)
+    assert codes_and_scales / pairs == 1.125
+    assert nbytes >= codes_and_scales
+    # the per-chunk mean, scales and scratch add well under 1% on top
+    assert nbytes < codes_and_scales * 1.01
+    with pytest.raises(nv.Nvfp4Error):
+        nv.kv_cache_bytes(24, 120, 8192, 16)  # head_dim % 16
+
+
+def _fake_tensor(rows, cols, layout=nv.SF_MMA, ptr=4096):
+    return nv.nvfp4_tensor(ptr, ptr, ptr, rows, cols, ((cols // 2 + 15) // 16) * 16,
+                           cols // 16 if layout == nv.SF_ROWMAJOR else 0, layout, 0)
+
+
+def test_host_argument_checks_return_before_any_device_work():
+    lib = nv.library()
+    t = _fake_tensor(16, 64)
+    # NULL input
+    assert lib.nvfp4_quantize(None, nv.BF16, 16, 64, 64, None, ctypes.byref(t), ctypes.c_void_p(4096),
+                              None) == nv.ERR_INVALID_ARG
+    # cols not a multiple of 16
+    bad = _fake_tensor(16, 64)
+    bad.cols = 40
+    assert lib.nvfp4_quantize(ctypes.c_void_p(4096), nv.BF16, 16, 40, 40, None, ctypes.byref(bad),
+                              ctypes.c_void_p(4096), None) == nv.ERR_SHAPE
+    # misaligned input pointer
+    assert lib.nvfp4_quantize(ctypes.c_void_p(4098), nv.BF16, 16, 64, 64, None, ctypes.byref(t),
+                              ctypes.c_void_p(4096), None) == nv.ERR_ALIGNMENT
+    # two-pass mode needs amax_out
+    assert lib.nvfp4_quantize(ctypes.c_void_p(4096), nv.BF16, 16, 64, 64, None, ctypes.byref(t), None,
+                              None) == nv.ERR_INVALID_ARG
+    # GEMM needs the tensor-core scale layout and matching K
+    a = _fake_tensor(16, 64, nv.SF_ROWMAJOR)
+    w = _fake_tensor(32, 64)
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(w), ctypes.c_void_p(4096), nv.FP32, 32, None,
+                          None) == nv.ERR_INVALID_ARG
+    a = _fake_tensor(16, 64)
+    w = _fake_tensor(32, 128)
+    assert lib.nvfp4_gemm(ctypes.byref(a), ctypes.byref(w), ctypes.c_void_p(4096), nv.FP32, 32, None,
+                          None) == nv.ERR_SHAPE
+    # KV cache init: misaligned memory, too small
+    h = nv.nvfp4_kv_cache()
+    assert lib.nvfp4_kv_cache_init(ctypes.c_void_p(4097), 1 << 30, 2, 16, 64, 2, ctypes.byref(h)) == \
+        nv.ERR_ALIGNMENT
+    assert lib.nvfp4_kv_cache_init(ctypes.c_void_p(4096), 16, 2, 16, 64, 2, ctypes.byref(h)) == nv.ERR_SHAPE
+    assert lib.nvfp4_kv_cache_init(ctypes.c_void_p(4096), 1 << 30, 2, 16, 64, 2, ctypes.byref(h)) == nv.OK
+    # append: wrong token count, slot out of range; window: empty list
+    assert lib.kv_quant_append(ctypes.byref(h), ctypes.c_void_p(4096), ctypes.c_void_p(4096), 63, 0,
+                               None) == nv.ERR_SHAPE
+    assert lib.kv_quant_append(ctypes.byref(h), ctypes.c_void_p(4096), ctypes.c_void_p(4096), 64, 2,
+                               None) == nv.ERR_INVALID_ARG
+    slots = (ctypes.c_int32 * 1)(5)
+    assert lib.kv_dequant_window(ctypes.byref(h), slots, 1, ctypes.c_void_p(4096),
+                                 ctypes.c_void_p(4096), None) == nv.ERR_INVALID_ARG
+    assert lib.kv_dequant_window(ctypes.byref(h), slots, 0, ctypes.c_void_p(4096),
+                                 ctypes.c_void_p(4096), None) == nv.ERR_INVALID_ARG

@@ -1,0 +1,171 @@
+"""GPU parity of nvfp4_gemm against the oracle: every FP32 output within
+1e-5 * sum_k |a_k w_k| of the float64 product of the exactly decoded operands
+(the tolerance of the benchmark spec), outputs with a zero bound exactly 0; the
+fused GELU + NVFP4 requantization epilogue checked step by step."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_w4a4_quantized_amax_b200 as nv
+import oracle
+import synth
+from gpu_helpers import canonical, dev_bf16, device_status, gpu_quantize, host_bits
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-5
+
+
+def gemm_case(a_bits, w_bits, out_bf16=False, rows=None):
+    qa, _ = gpu_quantize(a_bits, nv.SF_MMA)
+    qw, _ = gpu_quantize(w_bits, nv.SF_MMA)
+    M, N = a_bits.shape[0], w_bits.shape[0]
+    c = torch.full((M, N), float("nan"), dtype=torch.bfloat16 if out_bf16 else torch.float32,
+                   device="cuda")
+    nv.nvfp4_gemm(qa, qw, c)
+    torch.cuda.synchronize()
+    ac, asc, ag = canonical(qa)
+    wc, wsc, wg = canonical(qw)
+    ref, bound = oracle.gemm_ref(ac, asc, ag, wc, wsc, wg, rows=rows)
+    got = c.float().cpu().numpy().astype(np.float64)
+    if rows is not None:
+        got = got[rows]
+    return got, ref, bound, (qa, qw)
+
+
+def assert_within_bound(got, ref, bound, extra_rel=0.0):
+    err = np.abs(got - ref)
+    lim = TOL * bound + extra_rel * np.abs(ref)
+    bad = np.argwhere(err > lim)
+    assert bad.size == 0, (f"{len(bad)} outputs outside the bound; worst ratio "
+                           f"{float(np.max(err / np.maximum(bound, 1e-300))):.3e}")
+    zero = bound == 0
+    assert np.all(got[zero] == 0)
+
+
+def test_tiny_linear_128x256x512(cuda_dev):
+    a, w = synth.tiny_linear(0)
+    got, ref, bound, _ = gemm_case(a, w)
+    assert_within_bound(got, ref, bound)
+    assert device_status() == nv.OK
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 16, 16), (300, 272, 400), (129, 144, 1040), (64, 512, 3072),
+                                   (513, 256, 256)])
+def test_ragged_shapes(cuda_dev, M, N, K):
+    a = synth.activations(21, M, K)
+    w = synth.weights(21, 0, N, K)
+    got, ref, bound, _ = gemm_case(a, w)
+    assert_within_bound(got, ref, bound)
+
+
+def test_bf16_output(cuda_dev):
+    a = synth.activations(22, 200, 512)
+    w = synth.weights(22, 0, 384, 512)
+    got, ref, bound, _ = gemm_case(a, w, out_bf16=True)
+    # the bf16 store adds one rounding of the FP32 result (half an ulp at 8 bits)
+    assert_within_bound(got, ref, bound, extra_rel=2.0 ** -8)
+
+
+def test_zero_rows_and_columns_are_exact(cuda_dev):
+    a = synth.activations(23, 130, 256)
+    w = synth.weights(23, 0, 160, 256)
+    a[5] = 0
+    w[17] = 0x8000
+    got, ref, bound, _ = gemm_case(a, w)
+    assert np.all(got[5] == 0) and np.all(got[:, 17] == 0)
+    assert_within_bound(got, ref, bound)
+
+
+@pytest.mark.slow
+@pytest.mark.parametrize("K,N", [(3072, 3072), (3072, 9216), (3072, 14336), (14336, 3072)])
+def test_full_size_block_gemms_sampled_rows(cuda_dev, K, N):
+    """M = 8192 tokens: activations 0.5 * t3 with picked channels x30, weights
+    N(0, 0.02).  Rows sampled across every 128-row tile, all N columns each."""
+    a = synth.activations(2, 8192, K)
+    w = synth.weights(2, {3072: 0, 9216: 1, 14336: 2}[N] if K == 3072 else 3, N, K)
+    rows = np.unique(np.concatenate([np.arange(0, 8192, 97), [8191]]))
+    got, ref, bound, _ = gemm_case(a, w, rows=rows)
+    assert_within_bound(got, ref, bound)
+
+
+def fused_case(M, N, K, seed):
+    x = synth.activations(seed, M, K)
+    w1 = synth.weights(seed, 0, N, K)
+    qx, _ = gpu_quantize(x, nv.SF_MMA)
+    qw, _ = gpu_quantize(w1, nv.SF_MMA)
+    # plain GEMM: the FP32 pre-activation c
+    c = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    nv.nvfp4_gemm(qx, qw, c)
+    # calibration call: max|h| of this very input gives the supplied scale
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    h = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    nv.nvfp4_gemm(qx, qw, None, act=nv.ACT_GELU_TANH, h_out=h, q_amax_out=amax)
+    g_h = np.float32(amax.item()) / np.float32(2688.0)
+    q_h = nv.NVFP4Tensor(M, N, nv.SF_MMA)
+    q_h.scales.fill_(0x7F)  # padding must be overwritten with zeros
+    gin = torch.tensor([g_h], dtype=torch.float32, device="cuda")
+    amax2 = torch.zeros(1, dtype=torch.float32, device="cuda")
+    h2 = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    nv.nvfp4_gemm(qx, qw, None, act=nv.ACT_GELU_TANH, q_out=q_h, q_gscale_in=gin,
+                  q_amax_out=amax2, h_out=h2)
+    torch.cuda.synchronize()
+    return c.cpu().numpy(), h2.cpu().numpy(), q_h, float(g_h), float(amax2.item()), h.cpu().numpy()
+
+
+def test_fused_gelu_requant_epilogue(cuda_dev):
+    M, N, K = 300, 512, 384
+    c, h, q_h, g_h, amax_h, h_cal = fused_case(M, N, K, 24)
+    # (i) h is GELU(c) to within a few ulp of the float64 formula
+    ref_h = oracle.gelu_tanh(c)
+    err = np.abs(h.astype(np.float64) - ref_h)
+    assert np.all(err <= 8 * 2.0 ** -24 * (np.abs(c) + np.abs(ref_h)) + 1e-37)
+    assert np.array_equal(h, h_cal)  # deterministic
+    # (ii) codes and scales are the oracle's quantization of the GPU's own h with the supplied g
+    ref_q = oracle.quantize(h, gscale=g_h)
+    codes, scales, g = canonical(q_h)
+    assert g == g_h
+    assert np.array_equal(scales, ref_q.scales)
+    assert np.array_equal(codes, ref_q.codes)
+    raw = q_h.scales.cpu().numpy()
+    nb = N // 16
+    used = np.zeros(raw.size, bool)
+    used[[oracle.sf_mma_offset(r, j, N) for r in range(M) for j in range(nb)]] = True
+    assert np.all(raw[~used] == 0)
+    # (iii) the reported amax is max|h|
+    assert amax_h == float(np.abs(h).max())
+
+
+@pytest.mark.slow
+def test_fused_ffn_chunk_decomposed(cuda_dev):
+    """X 8192 x 3072 -> GEMM to 14336 + GELU + NVFP4 requant -> GEMM to 3072 (bf16).
+    Checked by parts on sampled rows: requant bit-exact on the GPU's own h, the
+    second GEMM within the bound on the GPU's NVFP4 intermediate."""
+    M, K, N = 8192, 3072, 14336
+    x = synth.activations(4, M, K)
+    w1 = synth.weights(4, 0, N, K)
+    w2 = synth.weights(4, 1, K, N)
+    qx, _ = gpu_quantize(x, nv.SF_MMA)
+    q1, _ = gpu_quantize(w1, nv.SF_MMA)
+    q2, _ = gpu_quantize(w2, nv.SF_MMA)
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    nv.nvfp4_gemm(qx, q1, None, act=nv.ACT_GELU_TANH, q_amax_out=amax,
+                  h_out=torch.empty((M, N), dtype=torch.float32, device="cuda"))
+    g_h = float(np.float32(amax.item()) / np.float32(2688.0))
+    q_h = nv.NVFP4Tensor(M, N, nv.SF_MMA)
+    h = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    nv.nvfp4_gemm(qx, q1, None, act=nv.ACT_GELU_TANH, q_out=q_h,
+                  q_gscale_in=torch.tensor([g_h], device="cuda"), h_out=h)
+    y = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    nv.nvfp4_gemm(q_h, q2, y)
+    torch.cuda.synchronize()
+    rows = np.arange(0, M, 211)
+    hs = h.cpu().numpy()[rows]
+    ref_q = oracle.quantize(hs, gscale=g_h)
+    codes, scales, _ = canonical(q_h)
+    assert np.array_equal(codes[rows], ref_q.codes)
+    assert np.array_equal(scales[rows], ref_q.scales)
+    c2, s2, g2 = canonical(q2)
+    ref, bound = oracle.gemm_ref(codes, scales, g_h, c2, s2, g2, rows=rows)
+    got = y.float().cpu().numpy()[rows].astype(np.float64)
+    assert_within_bound(got, ref, bound, extra_rel=2.0 ** -8)

@@ -1,0 +1,110 @@
+"""GPU parity of the NVFP4 KV cache against the oracle: per-(head, dim) mean,
+tensor scales, codes and scales of K' and V bit for bit after each append, and the
+multi-chunk window dequantization bit for bit."""
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_w4a4_quantized_amax_b200 as nv
+import oracle
+import synth
+from gpu_helpers import dev_bf16, device_status, host_bits
+
+pytestmark = pytest.mark.gpu
+
+
+def check_slot(cache, slot, ref):
+    kc, ks, vc, vs, mu, g = cache.slot_views(slot)
+    T, H, Dh = ref.T, ref.H, ref.Dh
+    assert np.array_equal(mu.cpu().numpy().view(np.uint32), ref.mu.view(np.uint32)), "mu"
+    gk, gv = g.cpu().numpy().tolist()
+    assert gk == ref.g_k and gv == ref.g_v
+    assert np.array_equal(ks.cpu().numpy(), ref.k_scales.ravel()), "K scales"
+    assert np.array_equal(kc.cpu().numpy(), ref.k_codes.ravel()), "K codes"
+    assert np.array_equal(vs.cpu().numpy(), ref.v_scales.ravel()), "V scales"
+    assert np.array_equal(vc.cpu().numpy(), ref.v_codes.ravel()), "V codes"
+
+
+def run_cache(heads, head_dim, T, chunks, window, seed, full_window_check=True, plant=None):
+    off = synth.kv_offsets(seed, heads, head_dim)
+    cache = nv.KVCache(heads, head_dim, T, chunks)
+    refs = []
+    for c in range(chunks):
+        k, v = synth.kv_chunk(seed, c, T, heads, head_dim, off)
+        if plant is not None:
+            plant(c, k, v)
+        nv.kv_quant_append(cache, dev_bf16(k), dev_bf16(v), c)
+        ref = oracle.kv_append(k, v)
+        torch.cuda.synchronize()
+        check_slot(cache, c, ref)
+        refs.append(ref)
+    assert device_status() == nv.OK
+    slots = list(range(chunks - window, chunks))
+    C = heads * head_dim
+    ko = torch.empty((window * T, heads, head_dim), dtype=torch.bfloat16, device="cuda")
+    vo = torch.empty_like(ko)
+    nv.kv_dequant_window(cache, slots, ko, vo)
+    kh, vh = host_bits(ko), host_bits(vo)
+    for i, s in enumerate(slots if full_window_check else slots[-1:]):
+        i = slots.index(s)
+        rk, rv = oracle.kv_dequant_chunk(refs[s])
+        assert np.array_equal(kh[i * T:(i + 1) * T], rk), f"K^ window entry {i}"
+        assert np.array_equal(vh[i * T:(i + 1) * T], rv), f"V^ window entry {i}"
+    return cache, refs
+
+
+def test_small_cache_ragged_geometry(cuda_dev):
+    # C = 144 columns (not a multiple of the 256-column stats tile), T = 1000 tokens
+    # (not a power of two: the mean needs a correctly rounded division)
+    run_cache(heads=3, head_dim=48, T=1000, chunks=3, window=2, seed=3)
+
+
+def test_window_order_repeats_and_any_slot_list(cuda_dev):
+    cache, refs = run_cache(heads=2, head_dim=64, T=256, chunks=4, window=4, seed=8)
+    slots = [3, 0, 0, 2, 1]
+    T = 256
+    ko = torch.empty((len(slots) * T, 2, 64), dtype=torch.bfloat16, device="cuda")
+    vo = torch.empty_like(ko)
+    nv.kv_dequant_window(cache, slots, ko, vo)
+    kh, vh = host_bits(ko), host_bits(vo)
+    for i, s in enumerate(slots):
+        rk, rv = oracle.kv_dequant_chunk(refs[s])
+        assert np.array_equal(kh[i * T:(i + 1) * T], rk)
+        assert np.array_equal(vh[i * T:(i + 1) * T], rv)
+
+
+def test_wide_range_columns_take_the_exact_path(cuda_dev):
+    """Columns whose magnitudes span more binades than a double sum can hold exactly:
+    the mean must still equal the exactly rounded one."""
+    def plant(c, k, v):
+        flat = k.reshape(k.shape[0], -1)
+        flat[5, 7] = 0x7E80       # 8.5e37
+        flat[9, 7] = 0x0001       # smallest bf16 subnormal
+        flat[11, 7] = 0xFE80      # -8.5e37: cancels, leaving tiny terms
+        flat[3, 33] = 0x4F00      # 2^31
+        flat[4, 33] = 0x2F80      # 2^-32
+        flat[:, 40] = 0           # an all-zero column
+        flat[:, 41] = 0x3F80      # a constant column
+    run_cache(heads=2, head_dim=32, T=64, chunks=2, window=2, seed=4, plant=plant)
+
+
+def test_nonfinite_chunk_leaves_slot_unchanged(cuda_dev):
+    heads, dh, T = 2, 32, 64
+    off = synth.kv_offsets(1, heads, dh)
+    cache = nv.KVCache(heads, dh, T, 2)
+    k, v = synth.kv_chunk(1, 0, T, heads, dh, off)
+    nv.kv_quant_append(cache, dev_bf16(k), dev_bf16(v), 0)
+    ref = oracle.kv_append(k, v)
+    device_status(clear=True)
+    k2, v2 = synth.kv_chunk(1, 1, T, heads, dh, off)
+    v2[7, 1, 3] = 0x7F80  # +inf
+    nv.kv_quant_append(cache, dev_bf16(k2), dev_bf16(v2), 0)
+    assert device_status(clear=True) == nv.ERR_NONFINITE
+    check_slot(cache, 0, ref)
+
+
+@pytest.mark.slow
+def test_full_size_cache_24x128_8192_tokens(cuda_dev):
+    """24 heads x 128, chunks of 8192 tokens: 5 appends (every slot checked) and a
+    4-chunk window of 32768 tokens, all values compared."""
+    run_cache(heads=24, head_dim=128, T=8192, chunks=5, window=4, seed=3)
