@@ -321,6 +321,7 @@ struct EncParams {
   uint8_t* v_scales;
   float* gscale;      // slot's (g_K, g_V)
   const unsigned* words;
+  unsigned* status;
 };
 
 __device__ __forceinline__ void encode_block16(const float (&v)[16], float g, float d6,
@@ -347,7 +348,10 @@ __device__ __forceinline__ void encode_block16(const float (&v)[16], float g, fl
 }
 
 __global__ void __launch_bounds__(kEncThreads) kv_encode_kernel(EncParams p) {
-  if (p.words[2]) return;
+  if (p.words[2]) {  // a NaN or Inf in K or V: report it, leave the slot unchanged
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(p.status, kStatusNonfinite);
+    return;
+  }
   const float gk = __uint_as_float(p.words[1]) / 2688.0f;
   const float gv = __uint_as_float(p.words[0]) / 2688.0f;
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -468,7 +472,6 @@ int64_t kv_scratch_bytes(int32_t heads, int32_t head_dim, int64_t chunk_tokens) 
 
 cudaError_t launch_kv_append(const KVLayout& L, const void* k, const void* v, int32_t slot,
                              unsigned* status, cudaStream_t s) {
-  (void)status;
   const int64_t C = (int64_t)L.heads * L.head_dim;
   const int64_t T = L.chunk_tokens;
   Scratch sc = scratch_at(L.base + L.off_scratch, C);
@@ -510,13 +513,11 @@ cudaError_t launch_kv_append(const KVLayout& L, const void* k, const void* v, in
   ep.v_scales = L.base + L.off_v_scales + (int64_t)slot * L.slot_scales_bytes;
   ep.gscale = reinterpret_cast<float*>(L.base + L.off_gscale) + 2 * (int64_t)slot;
   ep.words = sc.words;
+  ep.status = status;
   const int64_t want = (ep.nblocks + kEncThreads - 1) / kEncThreads;
   const int64_t cap = (int64_t)sm_count() * 8;
   kv_encode_kernel<<<(unsigned)(want < cap ? want : cap), kEncThreads, 0, s>>>(ep);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-  // a non-finite input is reported through the sticky status word
-  return cudaSuccess;
+  return cudaGetLastError();
 }
 
 cudaError_t launch_kv_window(const KVLayout& L, const int32_t* slots, int32_t n_slots, void* k_out,
