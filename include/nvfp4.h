@@ -84,7 +84,8 @@ typedef enum { NVFP4_SF_ROWMAJOR = 0, NVFP4_SF_MMA = 1 } nvfp4_sf_layout;
  *   codes : rows * ld_codes bytes; ld_codes >= cols / 2, multiple of 16;
  *           base 16-byte aligned.
  *   scales: see nvfp4_sf_layout; base 16-byte aligned.
- *   gscale: one FP32 tensor scale g. */
+ *   gscale: one FP32 tensor scale g.
+ * An empty tensor (rows == 0) may pass NULL codes and scales. */
 typedef struct nvfp4_tensor {
   uint8_t* codes;
   uint8_t* scales;
@@ -105,7 +106,8 @@ nvfp4_status nvfp4_scales_bytes(int64_t rows, int64_t cols, int32_t sf_layout, s
  * [TW] §一 defines the format; [TW] §四 / [ZD] apply it to activations and weights.
  *   x        : device, row-major [rows, cols] of `xt` (NVFP4_BF16 or NVFP4_FP32),
  *              leading dimension ldx elements (ldx >= cols); base and row pitch
- *              16-byte aligned.
+ *              16-byte aligned; may be NULL when rows == 0 (then g = 0, or the
+ *              supplied g, and amax = 0).
  *   gscale_in: NULL  -> the tensor scale is computed from x: g = RN(amax / 2688)
  *                       (two passes over x). amax_out is then REQUIRED.
  *              !NULL -> device FP32 g used as given (one pass over x, e.g. a

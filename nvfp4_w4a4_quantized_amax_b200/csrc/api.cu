@@ -57,7 +57,8 @@ int64_t sf_mma_bytes(int64_t rows, int64_t cols) {
 
 // Checks common to every nvfp4_tensor argument.
 nvfp4_status check_tensor(const nvfp4_tensor* t) {
-  if (!t || !t->codes || !t->scales || !t->gscale) return NVFP4_ERR_INVALID_ARG;
+  if (!t || !t->gscale) return NVFP4_ERR_INVALID_ARG;
+  if (t->rows > 0 && (!t->codes || !t->scales)) return NVFP4_ERR_INVALID_ARG;  // empty: may be NULL
   if (t->reserved != 0) return NVFP4_ERR_INVALID_ARG;
   if (t->sf_layout != NVFP4_SF_ROWMAJOR && t->sf_layout != NVFP4_SF_MMA) return NVFP4_ERR_INVALID_ARG;
   if (t->rows < 0 || t->cols <= 0 || t->cols % 16 != 0) return NVFP4_ERR_SHAPE;
@@ -104,7 +105,7 @@ nvfp4_status nvfp4_scales_bytes(int64_t rows, int64_t cols, int32_t sf_layout, s
 nvfp4_status nvfp4_quantize(const void* x, int32_t xt, int64_t rows, int64_t cols, int64_t ldx,
                             const float* gscale_in, const nvfp4_tensor* out, float* amax_out,
                             nvfp4_stream_t stream) {
-  if (!x || !valid_dtype(xt)) return NVFP4_ERR_INVALID_ARG;
+  if ((!x && rows > 0) || !valid_dtype(xt)) return NVFP4_ERR_INVALID_ARG;
   nvfp4_status st = check_tensor(out);
   if (st != NVFP4_OK) return st;
   if (out->rows != rows || out->cols != cols || ldx < cols) return NVFP4_ERR_SHAPE;
