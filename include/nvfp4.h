@@ -214,6 +214,31 @@ nvfp4_status nvfp4_kv_cache_init(void* dev_mem, size_t bytes, int32_t heads, int
 nvfp4_status kv_quant_append(const nvfp4_kv_cache* cache, const void* k, const void* v,
                              int64_t tokens, int32_t slot, nvfp4_stream_t stream);
 
+/* kv_quant_append_noalloc — kv_quant_append for callers that cannot allocate
+ * device memory.  No counterpart on the pages: it is a library convenience.
+ * Some callers may not call cudaMalloc: a host framework that owns all device
+ * memory through its own pool (a library allocation behind its back breaks its
+ * accounting and fragments the pool), a real-time loop that must not stall on
+ * the device-wide synchronization that cudaMalloc and cudaFree can imply, or a
+ * plugin interface that hands a kernel only its input and output buffers.  This
+ * entry point allocates nothing and needs no scratch from the caller: the
+ * per-chunk column statistics live in one static device array of the library
+ * (about 5 MiB, present on every device that loads the library until the
+ * process exits), not in the cache's scratch region, which it never touches.
+ * Inputs and outputs are exactly those of kv_quant_append and the slot it writes
+ * is bit-identical.
+ *   Limit: heads * head_dim <= NVFP4_NOALLOC_MAX_COLUMNS, else NVFP4_ERR_SHAPE.
+ *   Set-up: the first call on a device looks up the array's device address for
+ *   that device (the device current at the call); make that first call before
+ *   any stream capture.
+ *   Sharing: every call on a device uses the same array and it keeps the last
+ *   call's contents; the call clears what must start at zero itself.  Calls whose
+ *   work overlaps on the GPU (other streams, other threads) race on the array:
+ *   issue them on one stream or serialize them. */
+#define NVFP4_NOALLOC_MAX_COLUMNS 4096
+nvfp4_status kv_quant_append_noalloc(const nvfp4_kv_cache* cache, const void* k, const void* v,
+                                     int64_t tokens, int32_t slot, nvfp4_stream_t stream);
+
 /* kv_dequant_window — dequantize the chunks listed in `slots_host` (a HOST array
  * of n_slots slot ids, 1 <= n_slots <= 64, repeats allowed, any order) in one
  * launch, writing bf16 [n_slots * chunk_tokens][heads][head_dim] to k_out and

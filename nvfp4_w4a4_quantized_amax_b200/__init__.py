@@ -62,7 +62,8 @@ class nvfp4_kv_cache(ctypes.Structure):
 
 EXPORTS = ["nvfp4_version", "nvfp4_status_string", "nvfp4_scales_bytes", "nvfp4_quantize",
            "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_cache_bytes", "nvfp4_kv_cache_init",
-           "kv_quant_append", "kv_dequant_window", "nvfp4_get_device_status"]
+           "kv_quant_append", "kv_quant_append_noalloc", "kv_dequant_window",
+           "nvfp4_get_device_status"]
 
 
 def library():
@@ -94,6 +95,8 @@ def library():
             lib.nvfp4_kv_cache_init.argtypes = [vp, ctypes.c_size_t, i32, i32, i64, i32, KV]
             lib.kv_quant_append.restype = i32
             lib.kv_quant_append.argtypes = [KV, vp, vp, i64, i32, vp]
+            lib.kv_quant_append_noalloc.restype = i32
+            lib.kv_quant_append_noalloc.argtypes = [KV, vp, vp, i64, i32, vp]
             lib.kv_dequant_window.restype = i32
             lib.kv_dequant_window.argtypes = [KV, ctypes.POINTER(ctypes.c_int32), i32, vp, vp, vp]
             lib.nvfp4_get_device_status.restype = i32
@@ -240,6 +243,15 @@ def kv_quant_append(cache: KVCache, k, v, slot: int, stream=None):
     """Quantize one chunk (bf16 [tokens, heads, head_dim]) of K and V into `slot`."""
     _check(library().kv_quant_append(ctypes.byref(cache.handle), _ptr(k), _ptr(v), k.shape[0], slot,
                                      _stream(stream)), "kv_quant_append")
+
+
+def kv_quant_append_noalloc(cache: KVCache, k, v, slot: int, stream=None):
+    """kv_quant_append without any caller-provided scratch: the library's static
+    per-device array holds the column statistics (heads * head_dim <= 4096).
+    For callers that may not allocate device memory; calls racing on the GPU
+    share that array, so issue them on one stream."""
+    _check(library().kv_quant_append_noalloc(ctypes.byref(cache.handle), _ptr(k), _ptr(v), k.shape[0],
+                                             slot, _stream(stream)), "kv_quant_append_noalloc")
 
 
 def kv_dequant_window(cache: KVCache, slots: Sequence[int], k_out, v_out, stream=None):

@@ -6,6 +6,9 @@
 #include "kernels.h"
 #include "nvfp4.h"
 
+static_assert(NVFP4_NOALLOC_MAX_COLUMNS == nvfp4::kNoAllocMaxColumns,
+              "header and library agree on the static scratch limit");
+
 // One status word per device (a module global: every device that loads the
 // library holds its own copy).  Kernels record the first data error here.
 __device__ unsigned nvfp4_device_status_word;
@@ -303,6 +306,22 @@ nvfp4_status kv_quant_append(const nvfp4_kv_cache* cache, const void* k, const v
   if ((st = current_device(&status)) != NVFP4_OK) return st;
   return cuda_status(nvfp4::launch_kv_append(L, k, v, slot, status,
                                              reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status kv_quant_append_noalloc(const nvfp4_kv_cache* cache, const void* k, const void* v,
+                                     int64_t tokens, int32_t slot, nvfp4_stream_t stream) {
+  nvfp4::KVLayout L;
+  nvfp4_status st = check_cache(cache, &L);
+  if (st != NVFP4_OK) return st;
+  if (!k || !v) return NVFP4_ERR_INVALID_ARG;
+  if (!aligned16(k) || !aligned16(v)) return NVFP4_ERR_ALIGNMENT;
+  if (tokens != cache->chunk_tokens) return NVFP4_ERR_SHAPE;
+  if (slot < 0 || slot >= cache->max_chunks) return NVFP4_ERR_INVALID_ARG;
+  if ((int64_t)cache->heads * cache->head_dim > NVFP4_NOALLOC_MAX_COLUMNS) return NVFP4_ERR_SHAPE;
+  unsigned* status = nullptr;
+  if ((st = current_device(&status)) != NVFP4_OK) return st;
+  return cuda_status(nvfp4::launch_kv_append_noalloc(L, k, v, slot, status,
+                                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t* slots_host,

@@ -49,6 +49,11 @@ struct KVLayout {
 int64_t kv_scratch_bytes(int32_t heads, int32_t head_dim, int64_t chunk_tokens);
 cudaError_t launch_kv_append(const KVLayout& c, const void* k, const void* v, int32_t slot,
                              unsigned* status, cudaStream_t s);
+// Same append, but the statistics scratch is a static device array of the library
+// (at most kNoAllocMaxColumns columns) instead of the cache's scratch region.
+constexpr int64_t kNoAllocMaxColumns = 4096;
+cudaError_t launch_kv_append_noalloc(const KVLayout& c, const void* k, const void* v, int32_t slot,
+                                     unsigned* status, cudaStream_t s);
 cudaError_t launch_kv_window(const KVLayout& c, const int32_t* slots, int32_t n_slots, void* k_out,
                              void* v_out, cudaStream_t s);
 

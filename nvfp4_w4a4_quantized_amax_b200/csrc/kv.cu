@@ -20,6 +20,8 @@
 // most 45 - ceil(log2 T) binades (every value is then a multiple of the smallest
 // value's last bit and no partial sum can exceed 53 bits); a column outside that
 // range is summed exactly with integer limbs by kv_mu_kernel itself.
+#include <mutex>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -543,6 +545,96 @@ cudaError_t launch_kv_window(const KVLayout& L, const int32_t* slots, int32_t n_
   const int64_t want = (p.nblocks + kEncThreads - 1) / kEncThreads;
   const int64_t cap = (int64_t)sm_count() * 8;
   kv_window_kernel<<<(unsigned)(want < cap ? want : cap), kEncThreads, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------- append without caller scratch
+// Statistics scratch of kv_quant_append_noalloc: one static array per device that
+// loads the library, sized for at most kNoAllocMaxColumns = heads * head_dim
+// columns (64 token splits x 20 bytes per column, plus three words): 5.0 MiB.
+// Host code must not use this name as an address; it asks the runtime for the
+// device address of the current device's copy once (kv_noalloc_scratch).
+static __device__ __align__(256) uint8_t g_kv_noalloc_scratch[
+    (kSplits * kNoAllocMaxColumns * 8) + 3 * (kSplits * kNoAllocMaxColumns * 4) + 256];
+
+static_assert(kSplits * kNoAllocMaxColumns * 8 % 256 == 0 && kSplits * kNoAllocMaxColumns * 4 % 256 == 0,
+              "scratch_at's 256-byte alignment must leave the static array's layout unpadded");
+
+namespace {
+std::mutex g_noalloc_mu;
+uint8_t* g_noalloc_ptr[64];
+}  // namespace
+
+// Device address of this device's static scratch array (looked up once per device,
+// with that device current).
+static cudaError_t kv_noalloc_scratch(uint8_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_kv_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_ptr[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = g_noalloc_ptr[dev];
+  return cudaSuccess;
+}
+
+cudaError_t launch_kv_append_noalloc(const KVLayout& L, const void* k, const void* v, int32_t slot,
+                                     unsigned* status, cudaStream_t s) {
+  const int64_t C = (int64_t)L.heads * L.head_dim;
+  const int64_t T = L.chunk_tokens;
+  if (C > kNoAllocMaxColumns) return cudaErrorInvalidValue;
+  uint8_t* scratch = nullptr;
+  cudaError_t e = kv_noalloc_scratch(&scratch);
+  if (e != cudaSuccess) return e;
+  Scratch sc = scratch_at(scratch, C);
+  // the words accumulate with atomics: they must start at zero on every call; the
+  // per-split statistics are fully rewritten by kv_stats_kernel
+  if ((e = cudaMemsetAsync(sc.words, 0, 3 * sizeof(unsigned), s)) != cudaSuccess) return e;
+
+  StatsParams sp;
+  sp.k = (const uint8_t*)k;
+  sp.v = (const uint8_t*)v;
+  sp.T = T;
+  sp.C = C;
+  sp.tokens_per_split = (T + kSplits - 1) / kSplits;
+  sp.sc = sc;
+  dim3 sgrid((unsigned)((C + kStatsCols - 1) / kStatsCols), kSplits);
+  kv_stats_kernel<<<sgrid, kStatsThreads, 0, s>>>(sp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  MuParams mp;
+  mp.k = (const uint8_t*)k;
+  mp.T = T;
+  mp.C = C;
+  mp.sc = sc;
+  mp.mu = reinterpret_cast<float*>(L.base + L.off_mu) + (int64_t)slot * C;
+  int lg = 0;
+  while ((1ll << lg) < T) ++lg;
+  mp.log2T_ceil = lg;
+  kv_mu_kernel<<<(unsigned)((C + kMuThreads - 1) / kMuThreads), kMuThreads, 0, s>>>(mp);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  EncParams ep;
+  ep.k = (const uint8_t*)k;
+  ep.v = (const uint8_t*)v;
+  ep.nblocks = T * C / 16;
+  ep.cblocks = FastDiv((uint32_t)(C / 16));
+  ep.mu = mp.mu;
+  ep.k_codes = L.base + L.off_k_codes + (int64_t)slot * L.slot_codes_bytes;
+  ep.v_codes = L.base + L.off_v_codes + (int64_t)slot * L.slot_codes_bytes;
+  ep.k_scales = L.base + L.off_k_scales + (int64_t)slot * L.slot_scales_bytes;
+  ep.v_scales = L.base + L.off_v_scales + (int64_t)slot * L.slot_scales_bytes;
+  ep.gscale = reinterpret_cast<float*>(L.base + L.off_gscale) + 2 * (int64_t)slot;
+  ep.words = sc.words;
+  ep.status = status;
+  const int64_t want = (ep.nblocks + kEncThreads - 1) / kEncThreads;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  kv_encode_kernel<<<(unsigned)(want < cap ? want : cap), kEncThreads, 0, s>>>(ep);
   return cudaGetLastError();
 }
 
