@@ -111,10 +111,10 @@ nvfp4_status nvfp4_quantize(const void* x, int32_t xt, int64_t rows, int64_t col
   if ((!x && rows > 0) || !valid_dtype(xt)) return NVFP4_ERR_INVALID_ARG;
   nvfp4_status st = check_tensor(out);
   if (st != NVFP4_OK) return st;
-  if (out->rows != rows || out->cols != cols || ldx < cols) return NVFP4_ERR_SHAPE;
+  if (out->rows != rows || out->cols != cols || (rows > 0 && ldx < cols)) return NVFP4_ERR_SHAPE;
   if (!gscale_in && !amax_out) return NVFP4_ERR_INVALID_ARG;
   const int64_t esz = xt == NVFP4_BF16 ? 2 : 4;
-  if (!aligned16(x) || (ldx * esz) % 16 != 0) return NVFP4_ERR_ALIGNMENT;
+  if (rows > 0 && (!aligned16(x) || (ldx * esz) % 16 != 0)) return NVFP4_ERR_ALIGNMENT;
   if ((amax_out && (reinterpret_cast<uintptr_t>(amax_out) & 3u)) ||
       (gscale_in && (reinterpret_cast<uintptr_t>(gscale_in) & 3u)))
     return NVFP4_ERR_ALIGNMENT;

@@ -13,11 +13,15 @@
 // Structure: one persistent CTA per SM, 6 warps.
 //   warp 0      TMA producer: A and W code tiles (128 B swizzle, 128 rows x 256
 //               values per stage) and the stage's scale atoms (bulk copies).
-//   warp 1      MMA issuer: tcgen05.cp moves the scale atoms to tensor memory,
-//               tcgen05.mma.kind::mxf4nvf4.block_scale (UE4M3, 16-value blocks,
-//               K = 64 per instruction) accumulates into tensor memory.
+//   warp 1      MMA issuer: tcgen05.mma.kind::mxf4nvf4.block_scale (UE4M3,
+//               16-value blocks, K = 64 per instruction) into tensor memory.
 //   warps 2..5  epilogue: tcgen05.ld of the accumulator (one row per thread),
 //               scaling, optional GELU and NVFP4 requantization, stores.
+//   warps 6..9  scale factors: each warp copies the stage's scale atoms from
+//               shared memory into its 32-lane quarter of tensor memory with
+//               tcgen05.st (the 4-way lane replication the block-scaled MMA reads).
+//               Doing this on the SM's load/store path keeps it off the tensor
+//               pipe, where tcgen05.cp copies serialize with the MMAs.
 // Two accumulator buffers in tensor memory let the epilogue of one tile overlap
 // the main loop of the next.  No TMA load uses cluster multicast.
 //
@@ -38,8 +42,9 @@ constexpr int kBKBytes = 128;      // per stage: 128 bytes of packed codes = 256
 constexpr int kKPerMma = 64;       // values per tcgen05.mma (32 bytes)
 constexpr int kStages = 4;
 constexpr int kAccStages = 2;
-constexpr int kThreads = 192;
-constexpr int kEpiWarp0 = 2;
+constexpr int kThreads = 320;     // 10 warps
+constexpr int kEpiWarp0 = 2;      // warps 2..5: epilogue
+constexpr int kSfWarp0 = 6;       // warps 6..9: scale factors to tensor memory
 constexpr int kTmemCols = 512;
 constexpr int kSfColBase = kAccStages * kBN;  // scale-factor columns follow the accumulators
 
@@ -196,12 +201,6 @@ __device__ __forceinline__ void mma_mxf4nvf4(uint32_t d_tmem, uint64_t adesc, ui
       : "memory");
 }
 
-// 32 lanes x 128 bits from shared memory, replicated into the four 32-lane
-// quarters of tensor memory: the layout the block-scaled MMA reads its scales from.
-__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(bar)
                : "memory");
@@ -222,6 +221,19 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+// 32 consecutive 32-bit columns of this thread's lane (warp-collective).
+__device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,"
+      "%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]),
+      "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]),
+      "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
 __device__ __forceinline__ float gelu_tanh(float c) {
   // 0.5 c (1 + tanh(sqrt(2/pi) (c + 0.044715 c^3)))
   const float u = 0.7978845608028654f * (c + 0.044715f * (c * c * c));
@@ -239,7 +251,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty_bar = full_bar + kStages;
   uint64_t* tfull_bar = empty_bar + kStages;
   uint64_t* tempty_bar = tfull_bar + kAccStages;
-  uint64_t* done_bar = tempty_bar + kAccStages;
+  uint64_t* sf_bar = tempty_bar + kAccStages;  // [kStages] scale factors in tensor memory
+  uint64_t* done_bar = sf_bar + kStages;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
@@ -254,6 +267,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(smem_u32(&tfull_bar[a]), 1);
       mbar_init(smem_u32(&tempty_bar[a]), 4 * 32);
     }
+    for (int st = 0; st < kStages; ++st) mbar_init(smem_u32(&sf_bar[st]), 4);
     mbar_init(smem_u32(done_bar), 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -329,7 +343,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1u;
-          if (!mbar_wait(smem_u32(&full_bar[s]), ph, abort_flag, limit)) {
+          // the scale warps saw this stage's TMA land and put its scales in tensor memory
+          if (!mbar_wait(smem_u32(&sf_bar[s]), ph, abort_flag, limit)) {
             ok = false;
             break;
           }
@@ -337,12 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int nvalid = (int)min((int64_t)4, p.num_k64 - ks * 4);
           uint8_t* st = smem + s * kStageBytes;
           const uint32_t a_addr = smem_u32(st), b_addr = smem_u32(st + kABytes);
-          const uint32_t sfa_addr = smem_u32(st + kABytes + kBBytes);
-          const uint32_t sfb_addr = sfa_addr + kSfaBytes;
           for (int k = 0; k < nvalid; ++k) {
             const uint32_t sf_col = tmem_base + kSfColBase + (s * 4 + k) * 8;
-            tmem_cp_32x128b_warpx4(sf_col, smem_desc(sfa_addr + k * 512, 0, 128, 0));
-            tmem_cp_32x128b_warpx4(sf_col + 4, smem_desc(sfb_addr + k * 512, 0, 128, 0));
             const uint64_t adesc = smem_desc(a_addr + k * 32, 16, 1024, 2);
             const uint64_t bdesc = smem_desc(b_addr + k * 32, 16, 1024, 2);
             mma_mxf4nvf4(d_tmem, adesc, bdesc, sf_col, sf_col + 4, (ks > 0 || k > 0) ? 1u : 0u);
@@ -359,6 +370,51 @@ __global__ void __launch_bounds__(kThreads, 1)
       // drain: all MMAs this thread issued complete before tensor memory is freed
       mma_commit(smem_u32(done_bar));
       mbar_wait_drain(smem_u32(done_bar), 0, limit);
+    }
+  } else if (warp >= kSfWarp0) {
+    // ------------------------------------------------------------ scale factors
+    // Tensor-memory scale layout of the block-scaled MMA: for MMA k of stage s,
+    // columns c = kSfColBase + (s*4 + k)*8 hold A's scales (c .. c+3) and W's
+    // (c+4 .. c+7); lane l of EVERY 32-lane quarter holds, in column c + j, the 4
+    // block scales of row l + 32 j.  A 512-byte scale atom in shared memory has
+    // exactly that content in its 16-byte line l, so lane l of each quarter loads
+    // line l of the 4 atoms of A and of W and stores them as 32 columns.
+    const int quarter = warp & 3;
+    const int64_t kstages = (p.num_k64 + 3) / 4;
+    uint32_t it = 0;
+    bool ok = true;
+    for (int64_t tile = blockIdx.x; tile < p.num_tiles && ok; tile += gridDim.x) {
+      for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1u;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&full_bar[s]), ph, abort_flag, limit))) {
+          ok = false;
+          break;
+        }
+        const int nvalid = (int)min((int64_t)4, p.num_k64 - ks * 4);
+        const uint8_t* sfa = smem + s * kStageBytes + kABytes + kBBytes;
+        const uint8_t* sfb = sfa + kSfaBytes;
+        uint32_t r[32];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+          if (k < nvalid) {
+            a = *reinterpret_cast<const uint4*>(sfa + k * 512 + lane * 16);
+            b = *reinterpret_cast<const uint4*>(sfb + k * 512 + lane * 16);
+          }
+          r[8 * k + 0] = a.x; r[8 * k + 1] = a.y; r[8 * k + 2] = a.z; r[8 * k + 3] = a.w;
+          r[8 * k + 4] = b.x; r[8 * k + 5] = b.y; r[8 * k + 6] = b.z; r[8 * k + 7] = b.w;
+        }
+        tmem_st_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + kSfColBase + s * 32, r);
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(smem_u32(&sf_bar[s]));
+      }
+    }
+    if (!ok) {
+      if (lane == 0) set_status(p.status, kStatusTimeout);
+      *abort_flag = 1;
     }
   } else {
     // ------------------------------------------------------------ epilogue
