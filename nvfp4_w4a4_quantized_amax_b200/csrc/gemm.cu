@@ -30,6 +30,8 @@
 // asynchronous work (bounded again) before it frees tensor memory and exits.
 #include <cuda.h>
 
+#include <cstring>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -54,7 +56,10 @@ constexpr int kSfaBytes = (kBM / 128) * 4 * 512;  // 4 atoms (one per 64-value g
 constexpr int kSfbBytes = (kBN / 128) * 4 * 512;
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
 static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
-constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
+// Output staging for TMA stores: per epilogue warp two 32-row x 128-byte buffers.
+constexpr int kStagingBytesPerWarp = 2 * 32 * 128;
+constexpr int kStagingBytes = 4 * kStagingBytesPerWarp;
+constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
@@ -157,6 +162,20 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Tiled TMA store of a shared-memory box to global memory (coordinates are
+// element column x, row y; rows and columns outside the tensor are not written).
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(src), "r"(x), "r"(y)
+               : "memory");
+}
+
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
+  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
+               : "memory");
+}
+
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
@@ -243,10 +262,11 @@ __device__ __forceinline__ float gelu_tanh(float c) {
 // ----------------------------------------------------------------- the kernel
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w,
-                Params p) {
+                const __grid_constant__ CUtensorMap map_c, Params p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* bar_area = smem + kStages * kStageBytes;
+  uint8_t* staging = smem + kStages * kStageBytes;  // 1024-aligned
+  uint8_t* bar_area = staging + kStagingBytes;
   uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);
   uint64_t* empty_bar = full_bar + kStages;
   uint64_t* tfull_bar = empty_bar + kStages;
@@ -428,7 +448,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (blockIdx.x == 0 && threadIdx.x == kEpiWarp0 * 32) *p.q_gscale_out = gq;
     }
     unsigned amax_bits = 0;
-    uint32_t tcount = 0;
+    uint32_t tcount = 0, chunk = 0;
     for (int64_t tile = blockIdx.x; tile < p.num_tiles; tile += gridDim.x, ++tcount) {
       const int a = tcount % kAccStages;
       const uint32_t aph = (tcount / kAccStages) & 1u;
@@ -448,66 +468,70 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + a * kBN + cc;
         tmem_ld_32x32b_x32(taddr, r);
         const int64_t col0 = nt * kBN + cc;
-        if (!row_ok || col0 >= p.N) {
-          if (p.q_codes && !row_ok && col0 < p.N) {
-            // zero the scale padding of rows beyond M so the next GEMM reads finite scales
-            const int64_t j = col0 / 16;
-            if (row < (p.M + 127) / 128 * 128)
-              *reinterpret_cast<uint16_t*>(p.q_scales + sf_mma_offset(row, j, p.q_groups)) = 0;
-          }
-          continue;
-        }
+        if (col0 >= p.N) continue;  // warp-uniform
         float v[32];
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * gab;
-        if (col0 + 32 > p.N) {  // ragged last chunk (N % 32 == 16); never with q_codes
-          const int nv = (int)(p.N - col0);
-          for (int i = 0; i < nv; ++i) {
-            const float hv = p.act == 1 ? gelu_tanh(v[i]) : v[i];
-            if (p.c) {
-              if (p.c_bf16)
-                reinterpret_cast<uint16_t*>(p.c)[row * p.ldc + col0 + i] =
-                    (uint16_t)(pack_bf16x2(hv, 0.0f) & 0xFFFFu);
-              else
-                reinterpret_cast<float*>(p.c)[row * p.ldc + col0 + i] = hv;
-            }
-            if (p.h_out) p.h_out[row * p.N + col0 + i] = hv;
-            if (p.q_amax_out) amax_bits = max(amax_bits, __float_as_uint(hv) & 0x7FFFFFFFu);
-          }
-          continue;
-        }
         if (p.act == 1) {
 #pragma unroll
           for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
         }
         if (p.c) {
-          uint8_t* dst = p.c + (row * p.ldc + col0) * (p.c_bf16 ? 2 : 4);
+          // Stage this warp's 32 rows x 32 columns in shared memory (swizzled like the
+          // tensor map, so the writes are bank-conflict free) and store the box with
+          // one TMA store: full-line global writes, rows >= M / columns >= N clipped.
+          const uint32_t buf = smem_u32(staging) + (uint32_t)((warp - kEpiWarp0) * kStagingBytesPerWarp) +
+                               (uint32_t)((chunk & 1) * 4096);
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+          __syncwarp();
           if (p.c_bf16) {
 #pragma unroll
-            for (int q = 0; q < 4; ++q)
-              stg_v4(dst + 16 * q, make_uint4(pack_bf16x2(v[8 * q], v[8 * q + 1]),
-                                              pack_bf16x2(v[8 * q + 2], v[8 * q + 3]),
-                                              pack_bf16x2(v[8 * q + 4], v[8 * q + 5]),
-                                              pack_bf16x2(v[8 * q + 6], v[8 * q + 7])));
+            for (int u = 0; u < 4; ++u)
+              st_shared_v4(buf + lane * 64 + ((u ^ ((lane >> 1) & 3)) * 16),
+                           make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                                      pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
+                                      pack_bf16x2(v[8 * u + 6], v[8 * u + 7])));
           } else {
 #pragma unroll
-            for (int q = 0; q < 8; ++q)
-              stg_v4(dst + 16 * q, make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                                              __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3])));
+            for (int u = 0; u < 8; ++u)
+              st_shared_v4(buf + lane * 128 + ((u ^ (lane & 7)) * 16),
+                           make_uint4(__float_as_uint(v[4 * u]), __float_as_uint(v[4 * u + 1]),
+                                      __float_as_uint(v[4 * u + 2]), __float_as_uint(v[4 * u + 3])));
           }
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&map_c, buf, (int32_t)col0, (int32_t)(mt * kBM + quarter * 32));
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          }
+          ++chunk;
         }
+        if (!row_ok) {
+          if (p.q_codes) {
+            // zero the scale padding of rows beyond M so the next GEMM reads finite scales
+            if (row < (p.M + 127) / 128 * 128)
+              *reinterpret_cast<uint16_t*>(p.q_scales + sf_mma_offset(row, col0 / 16, p.q_groups)) = 0;
+          }
+          continue;
+        }
+        const int nvc = (int)min((int64_t)32, p.N - col0);  // 16 on a ragged last chunk
         if (p.h_out) {
           float* hd = p.h_out + row * p.N + col0;
+          if (nvc == 32) {
 #pragma unroll
-          for (int q = 0; q < 8; ++q)
-            stg_v4(hd + 4 * q, make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
-                                          __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3])));
+            for (int q = 0; q < 8; ++q)
+              stg_v4(hd + 4 * q, make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                            __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3])));
+          } else {
+            for (int i = 0; i < nvc; ++i) hd[i] = v[i];
+          }
         }
         if (p.q_amax_out) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) amax_bits = max(amax_bits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+          for (int i = 0; i < 32; ++i)
+            if (i < nvc) amax_bits = max(amax_bits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
         }
-        if (p.q_codes) {
+        if (p.q_codes) {  // N % 64 == 0 here, so the chunk is whole
           uint32_t w[4];
           uint32_t sc[2];
 #pragma unroll
@@ -542,6 +566,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       amax_bits = warp_max_u32(amax_bits);
       if (lane == 0 && amax_bits) atomicMax(reinterpret_cast<unsigned*>(p.q_amax_out), amax_bits);
     }
+    // every TMA store of this warp has finished before the CTA exits
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
   }
 
   tc_fence_before();
@@ -586,6 +613,23 @@ bool make_code_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t kb
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over the output C [M, N] (row pitch ldc elements) for the epilogue's
+// TMA stores: 32 x 32 boxes, swizzled like the staging buffers (128 B rows for
+// FP32, 64 B rows for bf16).
+bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t ld, bool bf16) {
+  EncodeTiledFn fn = get_encode_fn();
+  if (!fn) return false;
+  const int64_t esz = bf16 ? 2 : 4;
+  cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)(ld * esz)};
+  cuuint32_t box[2] = {32, 32};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides,
+            box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 }  // namespace
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
@@ -622,6 +666,9 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
   CUtensorMap ma, mw;
   if (!make_code_map(&ma, g.a.codes, g.M, g.K / 2, g.a.ld_codes, kBM)) return cudaErrorInvalidValue;
   if (!make_code_map(&mw, g.w.codes, g.N, g.K / 2, g.w.ld_codes, kBN)) return cudaErrorInvalidValue;
+  CUtensorMap mc;
+  memset(&mc, 0, sizeof(mc));
+  if (g.c && !make_out_map(&mc, g.c, g.M, g.N, g.ldc, g.c_bf16)) return cudaErrorInvalidValue;
 
   if (g.q_amax_out) {
     cudaError_t e = cudaMemsetAsync(g.q_amax_out, 0, sizeof(float), s);
@@ -637,7 +684,7 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
   cudaGetDevice(&dev);
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   const int grid = (int)(p.num_tiles < sms ? p.num_tiles : sms);
-  gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mw, p);
+  gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mw, mc, p);
   return cudaGetLastError();
 }
 
