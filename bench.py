@@ -514,6 +514,8 @@ def run_single_kernel(args):
             (lambda: nv.kv_dequant_window(cache, list(range(WINDOW)), ko, vo))
     else:
         raise SystemExit(f"unknown kernel {args.kernel}")
+    for _ in range(args.kernel_warmup):  # one-time launch setup stays out of the timed calls
+        fn()
     torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
@@ -539,6 +541,8 @@ def main():
                     help="profiling mode: gemm | gemm_fused | quantize | dequantize | kv_append | kv_window")
     ap.add_argument("--shape", default="8192,14336,3072", help="M,N,K for gemm; rows,cols for (de)quantize")
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--kernel-warmup", type=int, default=1,
+                    help="untimed calls before the timed ones in --kernel mode")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.kernel:

@@ -255,6 +255,15 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       : "memory");
 }
 
+__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
+      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
+      : "memory");
+}
+
 // GELU, tanh form: 0.5 c (1 + tanh(u)) with u = sqrt(2/pi) (c + 0.044715 c^3),
 // evaluated through the identity 0.5 (1 + tanh(u)) = 1 / (1 + exp(-2u)):
 //   h = c / (1 + 2^(-2 u log2(e)))
@@ -534,7 +543,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               stg_v4(hd + 4 * q, make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
                                             __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3])));
           } else {
-            for (int i = 0; i < nvc; ++i) hd[i] = v[i];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < nvc) hd[i] = v[i];
           }
         }
         if (p.q_amax_out) {
@@ -592,6 +603,402 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ============================================================ 2-CTA pair kernel
+// One cluster of 2 CTAs computes a 256 x 128 tile with tcgen05.mma.cta_group::2:
+// CTA r of the pair holds rows [128 r, 128 r + 128) of the A tile and rows
+// [64 r, 64 r + 64) of the W tile in its shared memory, and rows 128 r .. of the
+// accumulator in its tensor memory.  The even CTA issues every MMA; operands are
+// read from both CTAs' shared memory by the hardware.  Each CTA loads only its
+// own halves (no TMA multicast): 24 KB of codes per 256 K values per CTA for a
+// 128 x 128 share of the output, against 32 KB for a 128 x 128 tile of one CTA.
+//
+// Tensor memory per CTA (512 columns): accumulators 2 x 128, then one scale slot
+// per pipeline stage of 4 MMAs x 8 columns: [A scales 0..3 | W scales 4..7]; the
+// W scales of all 128 rows are present in both CTAs (the hardware reads them in
+// the SM that holds the accumulator rows).
+namespace pair {
+
+constexpr int kBM = 256;            // rows per pair tile (128 per CTA)
+constexpr int kBN = 256;            // columns per pair tile: 128 or 256
+constexpr int kBNHalf = kBN / 2;    // W rows per CTA
+constexpr int kWTiles = kBN / 128;  // 128-row W scale tiles per pair tile
+constexpr int kStages = 5;
+constexpr int kSfSlots = kStages;  // one per pipeline stage
+constexpr int kAccStages = kBN == 256 ? 1 : 2;
+constexpr int kEpiWarps = 16;  // 4 per tensor-memory lane quarter, 64 columns each
+constexpr int kEpiWarp0 = 2;
+constexpr int kSfWarp0 = kEpiWarp0 + kEpiWarps;
+constexpr int kThreads = 32 * (2 + kEpiWarps + 4);
+constexpr int kABytes = 128 * kBKBytes;           // 16 KB
+constexpr int kBBytes = kBNHalf * kBKBytes;       // 8 or 16 KB
+constexpr int kSfaBytes = 4 * 512;                // own 128 rows, 4 groups
+constexpr int kSfbBytes = kWTiles * 4 * 512;      // all kBN W rows of the tile x 4 groups
+constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
+static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
+constexpr int kStagingBytesPerWarp = 32 * 64;   // one output box: 32 rows x 64 bytes
+constexpr int kStagingBytes = kEpiWarps * kStagingBytesPerWarp;
+constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + 1024;
+static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
+static_assert(kBN == 4 * 64, "epilogue warps cover 64 columns each");
+constexpr int kSfColBase = kAccStages * kBN;      // 256
+constexpr int kSfPerMma = 4 + 4 * kWTiles;      // A's 4 columns, then 4 per W scale tile
+constexpr int kSfSlotCols = 4 * kSfPerMma;
+static_assert(kSfColBase + kSfSlots * kSfSlotCols <= 512, "tensor memory budget");
+static_assert(kBN == 128 || kBN == 256, "pair tile width");
+// kind::mxf4nvf4, E2M1 x E2M1, UE4M3 scales, K-major, N = kBN, M = 256
+constexpr uint32_t kIdesc2 = (1u << 7) | (1u << 10) | ((uint32_t)(kBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// address of the same shared-memory variable in CTA `rank` of the cluster
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(addr), "r"(rank));
+  return r;
+}
+
+// Arrive on a barrier of another CTA of the cluster.  What it orders is tensor
+// memory traffic, which the tcgen05 fences around the arrive and the wait order;
+// no cluster-scope memory fence is needed (and one costs a membar per arrive).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+  asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
+}
+
+__device__ __forceinline__ void mma2(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t sfa, uint32_t sfb,
+                                     uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(
+          d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc2), "r"(accumulate), "r"(sfa), "r"(sfb)
+      : "memory");
+}
+
+// arrive on the barrier at this shared-memory offset in every CTA of `mask`
+// once all previously issued MMAs of this thread have completed
+__device__ __forceinline__ void commit2(uint32_t bar, uint16_t mask) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 [%0], %1;" ::"r"(bar),
+      "h"(mask)
+      : "memory");
+}
+
+struct Params2 {
+  int64_t M, N, K;
+  int64_t num_m, num_n, num_k64, num_tiles;
+  int64_t a_row_tiles, w_row_tiles;  // 128-row scale tiles present in each scale buffer
+  int64_t sf_row_tile_bytes;         // num_k64 * 512
+  const uint8_t* sfa;
+  const uint8_t* sfw;
+  const float* ga;
+  const float* gw;
+  bool c_bf16;
+  unsigned* status;
+  unsigned long long wait_limit_ns;
+};
+
+// 22 warps: six share one of the SM's four 16K-register files, so at most
+// 16384 / (6 * 32) = 85 registers a thread (80 after allocation rounding).
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
+    gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w,
+                     const __grid_constant__ CUtensorMap map_c, Params2 p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* staging = smem + kStages * kStageBytes;
+  uint8_t* bar_area = staging + kStagingBytes;
+  uint64_t* full_bar = reinterpret_cast<uint64_t*>(bar_area);   // own TMA landed
+  uint64_t* empty_bar = full_bar + kStages;                      // MMAs of the stage done (both CTAs)
+  uint64_t* sf_bar = empty_bar + kStages;                        // leader: scales of both CTAs in TMEM
+  uint64_t* tfull_bar = sf_bar + kStages;                        // accumulator ready (both CTAs)
+  uint64_t* tempty_bar = tfull_bar + kAccStages;                 // leader: both epilogues drained
+  uint64_t* done_bar = tempty_bar + kAccStages;                  // leader: all MMAs complete
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_rank();
+  const bool leader = rank == 0;
+  const int64_t pair = blockIdx.x >> 1, num_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(smem_u32(&full_bar[s]), 1);
+      mbar_init(smem_u32(&empty_bar[s]), 1);
+      mbar_init(smem_u32(&sf_bar[s]), 2 * 4);
+    }
+    for (int a = 0; a < kAccStages; ++a) {
+      mbar_init(smem_u32(&tfull_bar[a]), 1);
+      mbar_init(smem_u32(&tempty_bar[a]), 2 * kEpiWarps);
+    }
+    mbar_init(smem_u32(done_bar), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(512)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  cluster_sync();  // barriers of both CTAs initialized, tensor memory allocated
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const unsigned long long limit = p.wait_limit_ns;
+  const int64_t kstages = (p.num_k64 + 3) / 4;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer (both CTAs)
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+      uint32_t it = 0;
+      bool ok = true;
+      for (int64_t tile = pair; tile < p.num_tiles && ok; tile += num_pairs) {
+        const int64_t mt = tile % p.num_m, nt = tile / p.num_m;
+        const int64_t a_rt = mt * 2 + rank;                 // this CTA's 128-row tile of A
+        const bool has_sfa = a_rt < p.a_row_tiles;
+        const int64_t n0 = nt * kBN;
+        const int64_t w_rt = n0 / 128;  // first 128-row W scale tile of the pair tile
+        int w_tiles = 0;                // W scale tiles present (the last pair tile may be ragged)
+        for (int t = 0; t < kWTiles; ++t) w_tiles += (w_rt + t < p.w_row_tiles) ? 1 : 0;
+        for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1u;
+          if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag, limit)) {
+            ok = false;
+            break;
+          }
+          const int64_t g0 = ks * 4;
+          const int nvalid = (int)min((int64_t)4, p.num_k64 - g0);
+          uint8_t* st = smem + s * kStageBytes;
+          const uint32_t fb = smem_u32(&full_bar[s]);
+          const uint32_t bytes = kABytes + kBBytes + (has_sfa ? nvalid * 512 : 0) + w_tiles * nvalid * 512;
+          mbar_arrive_expect_tx(fb, bytes);
+          tma_load_2d(smem_u32(st), &map_a, fb, (int32_t)(ks * kBKBytes), (int32_t)(mt * kBM + rank * 128));
+          tma_load_2d(smem_u32(st + kABytes), &map_w, fb, (int32_t)(ks * kBKBytes),
+                      (int32_t)(n0 + rank * kBNHalf));
+          if (has_sfa)
+            bulk_load(smem_u32(st + kABytes + kBBytes), p.sfa + a_rt * p.sf_row_tile_bytes + g0 * 512,
+                      nvalid * 512, fb);
+          for (int t = 0; t < w_tiles; ++t)
+            bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes + t * 2048),
+                      p.sfw + (w_rt + t) * p.sf_row_tile_bytes + g0 * 512, nvalid * 512, fb);
+        }
+      }
+      if (!ok) {
+        set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+      const uint32_t n_issued = it;
+      for (uint32_t j = (n_issued > (uint32_t)kStages ? n_issued - kStages : 0); j < n_issued; ++j)
+        mbar_wait_drain(smem_u32(&full_bar[j % kStages]), (j / kStages) & 1u, limit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer (leader CTA)
+    if (leader && lane == 0) {
+      uint32_t it = 0, tcount = 0;
+      bool ok = true;
+      for (int64_t tile = pair; tile < p.num_tiles && ok; tile += num_pairs, ++tcount) {
+        const int a = tcount % kAccStages;
+        const uint32_t aph = (tcount / kAccStages) & 1u;
+        if (!mbar_wait(smem_u32(&tempty_bar[a]), aph ^ 1u, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + a * kBN;
+        for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1u;
+          if (!mbar_wait(smem_u32(&sf_bar[s]), ph, abort_flag, limit)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nvalid = (int)min((int64_t)4, p.num_k64 - ks * 4);
+          uint8_t* st = smem + s * kStageBytes;
+          const uint32_t a_addr = smem_u32(st), b_addr = smem_u32(st + kABytes);
+          const uint32_t sf_slot = tmem_base + kSfColBase + s * kSfSlotCols;
+          // descriptors of MMA k: start address + 32 k bytes, i.e. + 2 k in the
+          // 16-byte address field (stage addresses stay far below its 2^18 bytes)
+          const uint64_t ad0 = smem_desc(a_addr, 16, 1024, 2), bd0 = smem_desc(b_addr, 16, 1024, 2);
+          if (nvalid == 4) {
+#pragma unroll
+            for (int k = 0; k < 4; ++k)
+              mma2(d_tmem, ad0 + 2 * k, bd0 + 2 * k, sf_slot + k * kSfPerMma, sf_slot + k * kSfPerMma + 4,
+                   (ks > 0 || k > 0) ? 1u : 0u);
+          } else {
+            for (int k = 0; k < nvalid; ++k)
+              mma2(d_tmem, ad0 + 2 * k, bd0 + 2 * k, sf_slot + k * kSfPerMma, sf_slot + k * kSfPerMma + 4,
+                   (ks > 0 || k > 0) ? 1u : 0u);
+          }
+          commit2(smem_u32(&empty_bar[s]), (uint16_t)0x3);
+        }
+        if (!ok) break;
+        commit2(smem_u32(&tfull_bar[a]), (uint16_t)0x3);
+      }
+      if (!ok) {
+        set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+      commit2(smem_u32(done_bar), (uint16_t)0x1);
+      mbar_wait_drain(smem_u32(done_bar), 0, limit);
+    }
+  } else if (warp >= kSfWarp0) {
+    // ------------------------------------------------------------ scale factors (both CTAs)
+    // Slot of stage s, MMA k (c = kSfPerMma k): columns c + 0..3 hold this CTA's A
+    // scales (lane l, column j: rows l + 32 j of its 128 rows), c + 4 .. c + 4 +
+    // 4 kWTiles - 1 the W scales of all kBN rows of the pair tile (lane l, column j:
+    // row l + 32 j).  Every group of 4 columns is line l of one of the stage's
+    // 512-byte scale atoms.  The slot is rewritten only after the stage's TMA landed
+    // again, i.e. after the MMAs that read it completed.
+    const int quarter = warp & 3;
+    const uint32_t leader_sf_bar0 = map_to_rank(smem_u32(&sf_bar[0]), 0);
+    uint32_t it = 0;
+    bool ok = true;
+    for (int64_t tile = pair; tile < p.num_tiles && ok; tile += num_pairs) {
+      const int64_t mt = tile % p.num_m, nt = tile / p.num_m;
+      const bool has_sfa = mt * 2 + rank < p.a_row_tiles;
+      const int64_t w_rt = nt * kBN / 128;
+      for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
+        const int s = it % kStages;
+        const uint32_t ph = (it / kStages) & 1u;
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&full_bar[s]), ph, abort_flag, limit))) {
+          ok = false;
+          break;
+        }
+        const int nvalid = (int)min((int64_t)4, p.num_k64 - ks * 4);
+        const uint8_t* sfa = smem + s * kStageBytes + kABytes + kBBytes;
+        const uint8_t* sfb = sfa + kSfaBytes;
+        uint32_t r[kSfSlotCols];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint4 a = make_uint4(0, 0, 0, 0);
+          if (k < nvalid && has_sfa) a = *reinterpret_cast<const uint4*>(sfa + k * 512 + lane * 16);
+          r[kSfPerMma * k + 0] = a.x; r[kSfPerMma * k + 1] = a.y;
+          r[kSfPerMma * k + 2] = a.z; r[kSfPerMma * k + 3] = a.w;
+#pragma unroll
+          for (int t = 0; t < kWTiles; ++t) {
+            uint4 b = make_uint4(0, 0, 0, 0);
+            if (k < nvalid && w_rt + t < p.w_row_tiles)
+              b = *reinterpret_cast<const uint4*>(sfb + t * 2048 + k * 512 + lane * 16);
+            r[kSfPerMma * k + 4 + 4 * t] = b.x; r[kSfPerMma * k + 5 + 4 * t] = b.y;
+            r[kSfPerMma * k + 6 + 4 * t] = b.z; r[kSfPerMma * k + 7 + 4 * t] = b.w;
+          }
+        }
+        const uint32_t slot = tmem_base + ((uint32_t)(quarter * 32) << 16) + kSfColBase + s * kSfSlotCols;
+        tmem_st_32x32b_x32(slot, *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
+        if constexpr (kSfSlotCols == 48) tmem_st_32x32b_x16(slot + 32, *reinterpret_cast<const uint32_t(*)[16]>(&r[32]));
+        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(leader_sf_bar0 + (uint32_t)(s * 8));
+      }
+    }
+    if (!ok) {
+      if (lane == 0) set_status(p.status, kStatusTimeout);
+      *abort_flag = 1;
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (both CTAs)
+    // Warp w reads tensor-memory lane quarter w % 4 (rows 32 (w % 4) .. + 31 of this
+    // CTA's 128) and columns [64 g, 64 g + 64), g = (w - kEpiWarp0) / 4.  It takes
+    // its 64 accumulator values into registers and frees the accumulator at once;
+    // the scaling and TMA stores then overlap the next tile's MMAs.
+    const int quarter = warp & 3;
+    const int cgroup = (warp - kEpiWarp0) / 4;
+    const uint32_t leader_tempty0 = map_to_rank(smem_u32(&tempty_bar[0]), 0);
+    const float gab = (*p.ga) * (*p.gw);
+    const uint32_t buf = smem_u32(staging) + (uint32_t)((warp - kEpiWarp0) * kStagingBytesPerWarp);
+    uint32_t tcount = 0;
+    for (int64_t tile = pair; tile < p.num_tiles; tile += num_pairs, ++tcount) {
+      const int a = tcount % kAccStages;
+      const uint32_t aph = (tcount / kAccStages) & 1u;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&tfull_bar[a]), aph, abort_flag, limit))) {
+        if (lane == 0) set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      uint32_t r[2][32];
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + a * kBN + cgroup * 64;
+      tmem_ld_32x32b_x32(taddr, r[0]);
+      tmem_ld_32x32b_x32(taddr + 32, r[1]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive_cluster(leader_tempty0 + (uint32_t)(a * 8));
+      const int64_t mt = tile % p.num_m, nt = tile / p.num_m;
+      const int32_t out_row = (int32_t)(mt * kBM + rank * 128 + quarter * 32);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int64_t col0 = nt * kBN + cgroup * 64 + h * 32;
+        if (col0 >= p.N) break;  // warp-uniform
+        float* v = reinterpret_cast<float*>(r[h]);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[h][i]) * gab;
+        // the staging box is free once the previous store has read it
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        __syncwarp();
+        if (p.c_bf16) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            st_shared_v4(buf + lane * 64 + ((u ^ ((lane >> 1) & 3)) * 16),
+                         make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                                    pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7])));
+          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&map_c, buf, (int32_t)col0, out_row);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          }
+        } else {
+          // FP32: two 32 x 16 boxes through the one staging box
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            if (b == 1) {
+              if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+              __syncwarp();
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              st_shared_v4(buf + lane * 64 + ((u ^ ((lane >> 1) & 3)) * 16),
+                           make_uint4(__float_as_uint(v[16 * b + 4 * u]), __float_as_uint(v[16 * b + 4 * u + 1]),
+                                      __float_as_uint(v[16 * b + 4 * u + 2]), __float_as_uint(v[16 * b + 4 * u + 3])));
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&map_c, buf, (int32_t)(col0 + 16 * b), out_row);
+              asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            }
+          }
+        }
+      }
+    }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  cluster_sync();  // no CTA leaves while its peer may still use its shared or tensor memory
+  tc_fence_after();
+  if (warp == 0) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512) : "memory");
+  }
+}
+
+}  // namespace pair
+
 // ----------------------------------------------------------------- host side
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -625,26 +1032,117 @@ bool make_code_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t kb
 }
 
 // 2-D map over the output C [M, N] (row pitch ldc elements) for the epilogue's
-// TMA stores: 32 x 32 boxes, swizzled like the staging buffers (128 B rows for
-// FP32, 64 B rows for bf16).
-bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t ld, bool bf16) {
+// TMA stores, boxes of 32 rows swizzled like the staging buffers: 32 columns
+// (128 B rows, 128-byte swizzle, FP32; 64 B rows, 64-byte swizzle, bf16), or with
+// `rows64` 64-byte rows for both types (16 FP32 or 32 bf16 columns).
+bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t ld, bool bf16,
+                  bool rows64 = false) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   const int64_t esz = bf16 ? 2 : 4;
+  const bool sw64 = bf16 || rows64;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * esz)};
-  cuuint32_t box[2] = {32, 32};
+  cuuint32_t box[2] = {(cuuint32_t)(sw64 ? 64 / esz : 32), 32};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            bf16 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+            sw64 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
 }  // namespace
 
+// Opt a kernel into its dynamic shared memory once per device.
+template <typename Kernel>
+cudaError_t set_smem_once(Kernel k, int bytes, bool (&done)[64]) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!done[dev]) {
+    e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    done[dev] = true;
+  }
+  return cudaSuccess;
+}
+
+int sm_count_gemm() {
+  int dev = 0, sms = 148;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s) {
+  pair::Params2 p;
+  p.M = g.M;
+  p.N = g.N;
+  p.K = g.K;
+  p.num_m = (g.M + pair::kBM - 1) / pair::kBM;
+  p.num_n = (g.N + pair::kBN - 1) / pair::kBN;
+  p.num_k64 = (g.K + kKPerMma - 1) / kKPerMma;
+  p.num_tiles = p.num_m * p.num_n;
+  p.a_row_tiles = (g.M + 127) / 128;
+  p.w_row_tiles = (g.N + 127) / 128;
+  p.sf_row_tile_bytes = p.num_k64 * 512;
+  p.sfa = g.a.scales;
+  p.sfw = g.w.scales;
+  p.ga = g.a.gscale;
+  p.gw = g.w.gscale;
+  p.c_bf16 = g.c_bf16;
+  p.status = g.status;
+  p.wait_limit_ns = kWaitLimitNs;
+
+  CUtensorMap ma, mw, mc;
+  if (!make_code_map(&ma, g.a.codes, g.M, g.K / 2, g.a.ld_codes, 128)) return cudaErrorInvalidValue;
+  if (!make_code_map(&mw, g.w.codes, g.N, g.K / 2, g.w.ld_codes, pair::kBNHalf)) return cudaErrorInvalidValue;
+  if (!make_out_map(&mc, g.c, g.M, g.N, g.ldc, g.c_bf16, true)) return cudaErrorInvalidValue;
+  static bool done[64];
+  cudaError_t e = set_smem_once(pair::gemm_pair_kernel, pair::kSmemBytes, done);
+  if (e != cudaSuccess) return e;
+  // Pairs must fit inside one GPC, so fewer than SMs / 2 of them may be resident
+  // at once; a persistent grid larger than that would run a second wave.
+  static int resident[64];
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (resident[dev] == 0) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(2 * (sm_count_gemm() / 2)), 1, 1);
+    cfg.blockDim = dim3(pair::kThreads, 1, 1);
+    cfg.dynamicSmemBytes = pair::kSmemBytes;
+    cfg.stream = s;
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeClusterDimension;
+    attr.val.clusterDim.x = 2;
+    attr.val.clusterDim.y = 1;
+    attr.val.clusterDim.z = 1;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    int n = 0;
+    e = cudaOccupancyMaxActiveClusters(&n, pair::gemm_pair_kernel, &cfg);
+    if (e != cudaSuccess) return e;
+    if (n <= 0) return cudaErrorInvalidConfiguration;
+    resident[dev] = n;
+  }
+  const int64_t max_pairs = resident[dev];
+  const int64_t pairs = p.num_tiles < max_pairs ? p.num_tiles : max_pairs;
+  pair::gemm_pair_kernel<<<(unsigned)(2 * pairs), pair::kThreads, pair::kSmemBytes, s>>>(ma, mw, mc, p);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
   if (g.M == 0 || g.N == 0) return cudaSuccess;
+  // Plain C output with at least one full pair tile of rows and columns: the
+  // CTA-pair kernel (256 x 256 tiles, one accumulator stage).  The fused GELU /
+  // requantization epilogue and small shapes: the single-CTA kernel, whose two
+  // accumulator stages overlap its heavier epilogue with the next tile's MMAs.
+  const bool plain = g.c != nullptr && g.act == 0 && g.q_codes == nullptr && g.h_out == nullptr &&
+                     g.q_amax_out == nullptr;
+  if (plain && g.M >= pair::kBM && g.N >= pair::kBN) return launch_gemm_pair(g, s);
   Params p;
   p.M = g.M;
   p.N = g.N;
@@ -685,15 +1183,10 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     cudaError_t e = cudaMemsetAsync(g.q_amax_out, 0, sizeof(float), s);
     if (e != cudaSuccess) return e;
   }
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  static bool done[64];
+  cudaError_t e = set_smem_once(gemm_kernel, kSmemBytes, done);
+  if (e != cudaSuccess) return e;
+  const int sms = sm_count_gemm();
   const int grid = (int)(p.num_tiles < sms ? p.num_tiles : sms);
   gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mw, mc, p);
   return cudaGetLastError();
