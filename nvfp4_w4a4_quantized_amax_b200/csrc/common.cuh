@@ -62,13 +62,21 @@ __device__ __forceinline__ uint32_t e4m3_from_float(float s) {
   return (uint32_t)(r & 0xFFu);
 }
 
-// Value of a non-negative E4M3 byte (never NaN here): exponent field 0 is the
-// subnormal range m * 2^-9; otherwise the fields map straight onto binary32.
+// Value of an E4M3 byte (never NaN here), through the exact E4M3 -> f16 -> f32
+// hardware conversions.
 __device__ __forceinline__ float e4m3_to_float(uint32_t b) {
-  const uint32_t e = (b >> 3) & 0xFu, m = b & 7u;
-  const float normal = __uint_as_float(((b & 0x7Fu) << 20) + (120u << 23));
-  const float sub = __int2float_rn((int)m) * 0.001953125f;  // exact
-  return e ? normal : sub;
+  uint32_t h2;
+  float f;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)b));
+  asm("cvt.f32.f16 %0, %1;" : "=f"(f) : "h"((uint16_t)(h2 & 0xFFFFu)));
+  return f;
+}
+
+// Hardware reciprocal approximation (at most 1 ulp from 1/x for normal x).
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
 }
 
 // ---------------------------------------------------------------- E2M1
@@ -115,46 +123,33 @@ __device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
   return r;
 }
 
-// Block encoder: D = RN(s * g) and rD = RN(1 / D) are computed once per block.
-// Fast path: q = RN(|x| * rD) is within 2 ulp of the exact quotient, so the
-// hardware RNE of q decides the code unless q lies within a few ulp of a number
-// whose binary32 fraction has only its top two bits set — every E2M1 midpoint is
-// such a number.  Groups holding such an element take the exact comparison path.
+// Block encoder: D = RN(s * g) and rD ~ 1 / D (hardware reciprocal, <= 1 ulp) are
+// computed once per block, and from rD two brackets rDlo < 1 / D < rDhi (rD scaled
+// by 1 -+ 2^-20, whose RN errors stay below 2^-23 + 2^-24).  For an element x the
+// exact quotient x / D then lies strictly between RN(x rDlo) and RN(x rDhi), and
+// E2M1 round-to-nearest-even (the hardware cvt, sign in bit 3 also for values
+// that round to zero) is monotonic: where both brackets give the same code it is
+// the code of the exact quotient.  Elements whose brackets differ (x / D within
+// ~2^-20 of an E2M1 midpoint, ties included) take the exact comparison path.
 struct BlockEncoder {
   float D, rD;
-  bool tiny;  // D < 2^-100: use the double comparison path for the whole block
+  bool tiny;  // D < 2^-100 or D > 2^125 (1/D near the flushed range): exact path for the whole block
+
+  float rDlo, rDhi;
 
   __device__ __forceinline__ BlockEncoder(float D_) : D(D_) {
-    rD = (D > 0.0f) ? 1.0f / D : 0.0f;
-    tiny = D < 7.8886090522101181e-31f;  // 2^-100
+    rD = (D > 0.0f) ? rcp_approx(D) : 0.0f;
+    rDlo = rD * 0.99999904632568359375f;  // 1 - 2^-20
+    rDhi = rD * 1.00000095367431640625f;  // 1 + 2^-20
+    tiny = D < 7.8886090522101181e-31f || D > 4.2535295865117308e37f;  // 2^-100, 2^125
   }
 
   __device__ __forceinline__ uint32_t index_slow(float ax) const {
     return tiny ? e2m1_index_exact_f64(ax, D) : e2m1_index_exact(ax, D);
   }
 
-  // 8 magnitudes -> 8 E2M1 indices packed into 32 bits (element k in bits 4k..4k+3)
-  __device__ __forceinline__ uint32_t encode8(const float (&ax)[8]) const {
-    if (!(D > 0.0f)) return 0u;
-    uint32_t word = 0;
-    bool any_slow = tiny;
-    float q[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      q[k] = ax[k] * rD;
-      const uint32_t u = __float_as_uint(q[k]);
-      const bool near = (((u + 4u) & 0x1FFFFFu) <= 8u) && q[k] > 0.125f && q[k] < 5.5f;
-      any_slow |= near;
-    }
-#pragma unroll
-    for (int k = 0; k < 8; k += 2) word |= e2m1x2_rn(q[k], q[k + 1]) << (4 * k);
-    if (any_slow) {
-      word = 0;
-#pragma unroll
-      for (int k = 0; k < 8; ++k) word |= index_slow(ax[k]) << (4 * k);
-    }
-    return word;
-  }
+  // 8 signed values -> 8 E2M1 codes packed into 32 bits (element k in bits 4k..4k+3)
+  __device__ __forceinline__ uint32_t encode8s(const float (&v)[8]) const;
 };
 
 // Per-block scale: s = E4M3_RNE_sat(RN(amax_b / d6)) with d6 = RN(6 g); d6 == 0 -> 0.
@@ -163,12 +158,56 @@ __device__ __forceinline__ uint32_t block_scale(float amax_b, float d6) {
   return e4m3_from_float(amax_b / d6);
 }
 
+// The same scale from the product t = RN(amax_b * r6), r6 = RN(1 / d6): t is within
+// 1.5 ulp of RN(amax_b / d6), so both round to the same E4M3 value unless an E4M3
+// rounding boundary lies within a few ulp of t.  In the normal range (t >= 2^-6)
+// those boundaries have binary32 fraction bits 19..0 = 0x80000 and are never a
+// power of two; t in the subnormal range, non-finite, or within 4 ulp of a
+// boundary takes the division.
+__device__ __forceinline__ uint32_t block_scale_fast(float amax_b, float d6, float r6) {
+  if (!(d6 > 0.0f)) return 0u;
+  const float t = amax_b * r6;
+  const uint32_t u = __float_as_uint(t);
+  if (!(t >= 0.015625f && t < 1.0e30f) || ((u + 0x80004u) & 0xFFFFFu) <= 8u) return e4m3_from_float(amax_b / d6);
+  return e4m3_from_float(t);
+}
+
 // Sign bits of 8 floats -> bit 3 of each nibble (so -0 encodes as 0x8).
 __device__ __forceinline__ uint32_t f32_signs8(const float (&v)[8]) {
   uint32_t r = 0;
 #pragma unroll
   for (int k = 0; k < 8; ++k) r |= (__float_as_uint(v[k]) >> 31) << (4 * k + 3);
   return r;
+}
+
+__device__ __forceinline__ uint32_t pack_e2m1x8(const float (&q)[8]) {
+  uint32_t word = 0;
+#pragma unroll
+  for (int k = 0; k < 8; k += 2) word |= e2m1x2_rn(q[k], q[k + 1]) << (4 * k);
+  return word;
+}
+
+__device__ __forceinline__ uint32_t BlockEncoder::encode8s(const float (&v)[8]) const {
+  if (!(D > 0.0f)) return f32_signs8(v);  // every magnitude index is 0
+  float ql[8], qh[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    ql[k] = v[k] * rDlo;
+    qh[k] = v[k] * rDhi;
+  }
+  uint32_t word = pack_e2m1x8(ql);
+  const uint32_t wh = pack_e2m1x8(qh);
+  if (tiny || word != wh) {
+    const uint32_t diff = tiny ? 0xFFFFFFFFu : (word ^ wh);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      if ((diff >> (4 * k)) & 0xFu) {
+        const uint32_t c = index_slow(fabsf(v[k])) | ((__float_as_uint(v[k]) >> 31) << 3);
+        word = (word & ~(0xFu << (4 * k))) | (c << (4 * k));
+      }
+    }
+  }
+  return word;
 }
 
 // Value of a 4-bit E2M1 code.

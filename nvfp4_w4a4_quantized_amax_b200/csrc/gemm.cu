@@ -461,10 +461,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int col_half = (warp - kEpiWarp0) / 4;  // columns [64 col_half, 64 col_half + 64) of a tile
     const int row_in_tile = quarter * 32 + lane;
     const float gab = (*p.ga) * (*p.gw);
-    float gq = 0.0f, d6q = 0.0f;
+    float gq = 0.0f, d6q = 0.0f, r6q = 0.0f;
     if (p.q_codes) {
       gq = *p.q_gscale_in;
       d6q = 6.0f * gq;
+      r6q = 1.0f / d6q;
       if (blockIdx.x == 0 && threadIdx.x == kEpiWarp0 * 32) *p.q_gscale_out = gq;
     }
     unsigned amax_bits = 0;
@@ -558,22 +559,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint32_t sc[2];
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
-            float ax[2][8], s0[8], s1[8];
+            float s0[8], s1[8];
             float amax_b = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-              ax[k / 8][k % 8] = fabsf(v[16 * b + k]);
-              amax_b = fmaxf(amax_b, ax[k / 8][k % 8]);
-            }
+            for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(v[16 * b + k]));
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               s0[k] = v[16 * b + k];
               s1[k] = v[16 * b + 8 + k];
             }
-            const uint32_t s = block_scale(amax_b, d6q);
+            const uint32_t s = block_scale_fast(amax_b, d6q, r6q);
             const BlockEncoder enc(e4m3_to_float(s) * gq);
-            w[2 * b] = enc.encode8(ax[0]) | f32_signs8(s0);
-            w[2 * b + 1] = enc.encode8(ax[1]) | f32_signs8(s1);
+            w[2 * b] = enc.encode8s(s0);
+            w[2 * b + 1] = enc.encode8s(s1);
             sc[b] = s;
           }
           stg_v4(p.q_codes + row * p.q_ld_codes + col0 / 2, make_uint4(w[0], w[1], w[2], w[3]));

@@ -326,25 +326,22 @@ struct EncParams {
   unsigned* status;
 };
 
-__device__ __forceinline__ void encode_block16(const float (&v)[16], float g, float d6,
+__device__ __forceinline__ void encode_block16(const float (&v)[16], float g, float d6, float r6,
                                                uint8_t* codes, uint8_t* scale) {
-  float ax[2][8], v0[8], v1[8];
+  float v0[8], v1[8];
   float amax_b = 0.0f;
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    ax[k / 8][k % 8] = fabsf(v[k]);
-    amax_b = fmaxf(amax_b, fabsf(v[k]));
-  }
+  for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(v[k]));
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
     v0[k] = v[k];
     v1[k] = v[8 + k];
   }
-  const uint32_t s = block_scale(amax_b, d6);
+  const uint32_t s = block_scale_fast(amax_b, d6, r6);
   const BlockEncoder enc(e4m3_to_float(s) * g);
   uint2 out;
-  out.x = enc.encode8(ax[0]) | f32_signs8(v0);
-  out.y = enc.encode8(ax[1]) | f32_signs8(v1);
+  out.x = enc.encode8s(v0);
+  out.y = enc.encode8s(v1);
   stg_v2(codes, out);
   *scale = (uint8_t)s;
 }
@@ -361,6 +358,7 @@ __global__ void __launch_bounds__(kEncThreads) kv_encode_kernel(EncParams p) {
     p.gscale[1] = gv;
   }
   const float d6k = 6.0f * gk, d6v = 6.0f * gv;
+  const float r6k = 1.0f / d6k, r6v = 1.0f / d6v;
   const int64_t stride = (int64_t)gridDim.x * kEncThreads;
   for (int64_t b = (int64_t)blockIdx.x * kEncThreads + threadIdx.x; b < p.nblocks; b += stride) {
     const uint32_t row = p.cblocks.div((uint32_t)b);
@@ -394,8 +392,8 @@ __global__ void __launch_bounds__(kEncThreads) kv_encode_kernel(EncParams p) {
         vv[2 * q + 1] = bf16_hi(w[q]);
       }
     }
-    encode_block16(kv, gk, d6k, p.k_codes + b * 8, p.k_scales + b);
-    encode_block16(vv, gv, d6v, p.v_codes + b * 8, p.v_scales + b);
+    encode_block16(kv, gk, d6k, r6k, p.k_codes + b * 8, p.k_scales + b);
+    encode_block16(vv, gv, d6v, r6v, p.v_codes + b * 8, p.v_scales + b);
   }
 }
 

@@ -97,6 +97,7 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(EncodeParams p) {
   }
   if (blockIdx.x == 0 && threadIdx.x == 0) *p.gscale_out = g;
   const float d6 = 6.0f * g;
+  const float r6 = 1.0f / d6;
 
   unsigned local_max = 0;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
@@ -129,19 +130,15 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(EncodeParams p) {
       }
     }
     float amax_b = 0.0f;
-    float ax[2][8];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      ax[k / 8][k % 8] = fabsf(v[k]);
-      amax_b = fmaxf(amax_b, ax[k / 8][k % 8]);
-    }
+    for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(v[k]));
     if (p.amax_accum) {
       unsigned bits = 0;
 #pragma unroll
       for (int k = 0; k < 16; ++k) bits = max(bits, __float_as_uint(v[k]) & 0x7FFFFFFFu);
       local_max = max(local_max, bits);
     }
-    const uint32_t s = block_scale(amax_b, d6);
+    const uint32_t s = block_scale_fast(amax_b, d6, r6);
     const BlockEncoder enc(e4m3_to_float(s) * g);
     float v0[8], v1[8];
 #pragma unroll
@@ -150,8 +147,8 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(EncodeParams p) {
       v1[k] = v[8 + k];
     }
     uint2 out;
-    out.x = enc.encode8(ax[0]) | f32_signs8(v0);
-    out.y = enc.encode8(ax[1]) | f32_signs8(v1);
+    out.x = enc.encode8s(v0);
+    out.y = enc.encode8s(v1);
     stg_v2(p.codes + (int64_t)r * p.ld_codes + (int64_t)j * 8, out);
     p.scales[soff] = (uint8_t)s;
   }

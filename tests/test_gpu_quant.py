@@ -59,6 +59,30 @@ def test_midpoints_ties_and_edges(cuda_dev):
         assert_quant_equal(q, oracle.quantize(x))
 
 
+def test_block_scale_rounding_boundaries(cuda_dev):
+    """Blocks whose max|x| / RN(6 g) lies exactly on, or one bf16 step either side
+    of, an E4M3 rounding boundary (every normal-range midpoint, the subnormal
+    midpoints and the saturation edge), with g = 2^-10 supplied so RN(6 g) is exact."""
+    rng = np.random.default_rng(7)
+    g = 2.0 ** -10
+    d6 = 6.0 * g
+    targets = [(1.0 + (2 * m + 1) / 16.0) * 2.0 ** e for e in range(-6, 9) for m in range(8)]
+    targets += [(j + 0.5) * 2.0 ** -9 for j in range(8)] + [448.0, 464.0, 480.0]
+    rows = []
+    for t in targets:
+        amax_bits = int(np.float32(t * d6).view(np.uint32) >> 16)
+        for delta in (-1, 0, 1):
+            top = np.array([(amax_bits + delta) << 16], np.uint32).view(np.float32)[0]
+            vals = (rng.uniform(-0.9, 0.9, 16) * top).astype(np.float32)
+            vals[rng.integers(16)] = top * rng.choice([-1.0, 1.0])
+            rows.append((vals.view(np.uint32) >> 16).astype(np.uint16))
+    x = np.stack(rows)
+    x = np.concatenate([x, np.zeros(((-len(x)) % 8, 16), np.uint16)]).reshape(-1, 128)
+    for layout in (nv.SF_ROWMAJOR, nv.SF_MMA):
+        q, _ = gpu_quantize(x, layout, gscale=g)
+        assert_quant_equal(q, oracle.quantize(x, gscale=g))
+
+
 @pytest.mark.parametrize("scale", [1e-30, 1e-36, 2.0 ** -133 * 7, 1e30, 3e38])
 def test_extreme_magnitudes(cuda_dev, scale):
     x = synth.activations(3, 16, 64)
@@ -87,6 +111,19 @@ def test_supplied_gscale_one_pass(cuda_dev):
         ref = oracle.quantize(x, gscale=gs)
         assert amax == ref.amax
         assert_quant_equal(q, ref)
+
+
+def test_supplied_gscale_huge_block_scales(cuda_dev):
+    """A supplied tensor scale large enough that D = s g exceeds 2^125 (so 1/D is
+    near the flushed range) with values near the top of the binary32 range."""
+    x = synth.activations(6, 64, 128)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64) * (3.0e38 / 30.0)
+    xf = np.clip(xf, -3.3e38, 3.3e38).astype(np.float32)
+    xb = (xf.view(np.uint32) >> 16).astype(np.uint16)
+    for gs in (1.0e37, 3.0e36, 2.0 ** 120):
+        gs = float(np.float32(gs))
+        q, _ = gpu_quantize(xb, nv.SF_MMA, gscale=gs)
+        assert_quant_equal(q, oracle.quantize(xb, gscale=gs))
 
 
 def test_all_zero_and_empty(cuda_dev):
