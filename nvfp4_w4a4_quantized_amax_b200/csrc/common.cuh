@@ -210,11 +210,33 @@ __device__ __forceinline__ uint32_t BlockEncoder::encode8s(const float (&v)[8]) 
   return word;
 }
 
-// Value of a 4-bit E2M1 code.
-__device__ __forceinline__ float e2m1_to_float(uint32_t c) {
-  // twice the magnitudes {0,0.5,1,1.5,2,3,4,6} = {0,1,2,3,4,6,8,12}, one nibble each
-  const float mag = __int2float_rn((int)((0xC8643210u >> (4 * (c & 7u))) & 0xFu)) * 0.5f;
-  return (c & 8u) ? -mag : mag;
+// E4M3 byte -> the same value in both halves of an f16x2 (exact conversion).
+__device__ __forceinline__ uint32_t e4m3_to_f16x2_bcast(uint32_t b) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)(b | (b << 8))));
+  return h2;
+}
+
+// Eight E2M1 codes (one 32-bit word, element k in bits 4k..4k+3) times a block
+// scale given as f16x2: four f16x2 products, element 2i in the low half of p[i].
+// The hardware E2M1 -> f16 conversion is exact, and so is the f16 product: the
+// magnitudes e2m1 * s lie in [2^-10, 6 * 448] with at most 6 significant bits.
+__device__ __forceinline__ void e2m1x8_times_scale(uint32_t w, uint32_t s2, uint32_t (&p)[4]) {
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t.reg .b32 h0, h1, h2, h3;\n\t"
+      "mov.b32 {b0, b1, b2, b3}, %4;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h0, b0;\n\tcvt.rn.f16x2.e2m1x2 h1, b1;\n\t"
+      "cvt.rn.f16x2.e2m1x2 h2, b2;\n\tcvt.rn.f16x2.e2m1x2 h3, b3;\n\t"
+      "mul.rn.f16x2 %0, h0, %5;\n\tmul.rn.f16x2 %1, h1, %5;\n\t"
+      "mul.rn.f16x2 %2, h2, %5;\n\tmul.rn.f16x2 %3, h3, %5;\n\t}"
+      : "=r"(p[0]), "=r"(p[1]), "=r"(p[2]), "=r"(p[3])
+      : "r"(w), "r"(s2));
+}
+
+// f16x2 -> its two halves as floats (exact).
+__device__ __forceinline__ void f16x2_to_f32x2(uint32_t h, float& lo, float& hi) {
+  asm("{\n\t.reg .b16 l, u;\n\tmov.b32 {l, u}, %2;\n\tcvt.f32.f16 %0, l;\n\tcvt.f32.f16 %1, u;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(h));
 }
 
 // Offset of block scale (r, j) in the tensor-core (MMA) scale layout.

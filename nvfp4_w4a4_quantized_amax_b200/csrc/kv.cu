@@ -30,8 +30,10 @@ namespace {
 
 constexpr int kStatsThreads = 256;   // 8 warps; each lane owns 8 consecutive columns
 constexpr int kStatsCols = 256;      // columns per CTA
-constexpr int kSplits = 64;          // token splits of the stats pass
-constexpr int kMuThreads = 256;
+constexpr int kSplits = 64;          // most token splits of the stats pass (scratch size)
+constexpr int kStatsUnroll = 4;      // token rows in flight per warp
+constexpr int kMuThreads = 256;      // 8 warps share the splits of kMuCols columns
+constexpr int kMuCols = 32;
 constexpr int kEncThreads = 256;
 constexpr int kMaxWindow = 64;
 
@@ -65,7 +67,7 @@ struct StatsParams {
   const uint8_t* k;
   const uint8_t* v;
   int64_t T, C;
-  int64_t tokens_per_split;
+  int64_t tokens_per_split;  // splits = gridDim.y
   Scratch sc;
 };
 
@@ -89,25 +91,37 @@ __global__ void __launch_bounds__(kStatsThreads) kv_stats_kernel(StatsParams p) 
   }
   unsigned kbad = 0, vmax = 0;
   if (active) {
-    for (int64_t t = t_begin + warp; t < t_end; t += kStatsThreads / 32) {
-      const uint4 kw = ldg_nc_v4(p.k + (t * p.C + c0) * 2);
-      const uint4 vw = ldg_nc_v4(p.v + (t * p.C + c0) * 2);
-      const uint32_t w[4] = {kw.x, kw.y, kw.z, kw.w};
+    constexpr int kRowStep = kStatsThreads / 32;
+    for (int64_t t0 = t_begin + warp; t0 < t_end; t0 += kRowStep * kStatsUnroll) {
+      uint4 kw[kStatsUnroll], vw[kStatsUnroll];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const uint32_t bits = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
-        const float f = __uint_as_float(bits << 16);
-        sum[i] += (double)f;
-        kmax[i] = fmaxf(kmax[i], f);
-        kmin[i] = fminf(kmin[i], f);
-        const unsigned a = (bits & 0x7FFFu) << 16;
-        kbad = max(kbad, a);
-        amin[i] = min(amin[i], a ? a : 0xFFFFFFFFu);
+      for (int u = 0; u < kStatsUnroll; ++u) {
+        const int64_t t = t0 + (int64_t)u * kRowStep;
+        if (t < t_end) {
+          kw[u] = ldg_nc_v4(p.k + (t * p.C + c0) * 2);
+          vw[u] = ldg_nc_v4(p.v + (t * p.C + c0) * 2);
+        }
       }
-      vmax = __vmaxu2(vmax, vw.x & 0x7FFF7FFFu);
-      vmax = __vmaxu2(vmax, vw.y & 0x7FFF7FFFu);
-      vmax = __vmaxu2(vmax, vw.z & 0x7FFF7FFFu);
-      vmax = __vmaxu2(vmax, vw.w & 0x7FFF7FFFu);
+#pragma unroll
+      for (int u = 0; u < kStatsUnroll; ++u) {
+        if (t0 + (int64_t)u * kRowStep >= t_end) break;
+        const uint32_t w[4] = {kw[u].x, kw[u].y, kw[u].z, kw[u].w};
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t bits = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
+          const float f = __uint_as_float(bits << 16);
+          sum[i] += (double)f;
+          kmax[i] = fmaxf(kmax[i], f);
+          kmin[i] = fminf(kmin[i], f);
+          const unsigned a = (bits & 0x7FFFu) << 16;
+          kbad = max(kbad, a);
+          amin[i] = min(amin[i], a ? a : 0xFFFFFFFFu);
+        }
+        vmax = __vmaxu2(vmax, vw[u].x & 0x7FFF7FFFu);
+        vmax = __vmaxu2(vmax, vw[u].y & 0x7FFF7FFFu);
+        vmax = __vmaxu2(vmax, vw[u].z & 0x7FFF7FFFu);
+        vmax = __vmaxu2(vmax, vw[u].w & 0x7FFF7FFFu);
+      }
     }
   }
   vmax = max(vmax >> 16, vmax & 0xFFFFu) << 16;
@@ -226,25 +240,60 @@ __device__ float mean_from_exact_double(double S, unsigned T) {
 struct MuParams {
   const uint8_t* k;
   int64_t T, C;
+  int nsplits;
   Scratch sc;
   float* mu;   // slot's mu [C]
   int log2T_ceil;
 };
 
+// kMuCols columns per CTA: warp w folds splits w, w + 8, ... of every column (lane
+// = column), warp 0 combines the 8 partial results.  When a column passes the
+// range test every partial sum is an exact double, so the order of the additions
+// does not matter.
 __global__ void __launch_bounds__(kMuThreads) kv_mu_kernel(MuParams p) {
   if (p.sc.words[2]) return;  // non-finite input: the slot stays unchanged
-  const int64_t c = (int64_t)blockIdx.x * kMuThreads + threadIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  constexpr int kWarps = kMuThreads / 32;
+  const int64_t c = (int64_t)blockIdx.x * kMuCols + lane;
+  __shared__ double r_sum[kWarps][kMuCols];
+  __shared__ float r_max[kWarps][kMuCols];
+  __shared__ float r_min[kWarps][kMuCols];
+  __shared__ unsigned r_amin[kWarps][kMuCols];
+  __shared__ int n_inexact;
+  __shared__ int inexact_cols[kMuCols];
+  __shared__ float inexact_mu[kMuCols];
+  __shared__ unsigned long long limbs[2][kLimbs];
+  if (threadIdx.x == 0) n_inexact = 0;
+  {
+    double S = 0.0;
+    float mx = -3.402823466e38f, mn = 3.402823466e38f;
+    unsigned am = 0xFFFFFFFFu;
+    if (c < p.C) {
+      for (int sp = warp; sp < p.nsplits; sp += kWarps) {
+        const int64_t o = (int64_t)sp * p.C + c;
+        S += p.sc.sum[o];
+        mx = fmaxf(mx, ordered_to_float(p.sc.kmax[o]));
+        mn = fminf(mn, ordered_to_float(p.sc.kmin[o]));
+        am = min(am, p.sc.amin[o]);
+      }
+    }
+    r_sum[warp][lane] = S;
+    r_max[warp][lane] = mx;
+    r_min[warp][lane] = mn;
+    r_amin[warp][lane] = am;
+  }
+  __syncthreads();
   double S = 0.0;
   float kmax = -3.402823466e38f, kmin = 3.402823466e38f;
   unsigned amin = 0xFFFFFFFFu;
   bool exact = true;
-  if (c < p.C) {
-    for (int sp = 0; sp < kSplits; ++sp) {
-      const int64_t o = (int64_t)sp * p.C + c;
-      S += p.sc.sum[o];
-      kmax = fmaxf(kmax, ordered_to_float(p.sc.kmax[o]));
-      kmin = fminf(kmin, ordered_to_float(p.sc.kmin[o]));
-      amin = min(amin, p.sc.amin[o]);
+  if (warp == 0 && c < p.C) {
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      S += r_sum[w][lane];
+      kmax = fmaxf(kmax, r_max[w][lane]);
+      kmin = fminf(kmin, r_min[w][lane]);
+      amin = min(amin, r_amin[w][lane]);
     }
     if (amin != 0xFFFFFFFFu) {
       const float amax = fmaxf(fabsf(kmax), fabsf(kmin));
@@ -252,18 +301,13 @@ __global__ void __launch_bounds__(kMuThreads) kv_mu_kernel(MuParams p) {
       const int e_min = max((int)((amin >> 23) & 0xFF), 1);
       exact = (e_max - e_min) <= 45 - p.log2T_ceil;
     }
+    if (!exact) inexact_cols[atomicAdd(&n_inexact, 1)] = lane;
   }
-  __shared__ int n_inexact;
-  __shared__ int inexact_cols[kMuThreads];
-  __shared__ float inexact_mu[kMuThreads];
-  __shared__ unsigned long long limbs[2][kLimbs];
-  if (threadIdx.x == 0) n_inexact = 0;
-  __syncthreads();
-  if (c < p.C && !exact) inexact_cols[atomicAdd(&n_inexact, 1)] = threadIdx.x;
   __syncthreads();
   // exact integer-limb sums for the (rare) columns outside the double's range
-  for (int i = 0; i < n_inexact; ++i) {
-    const int64_t cc = (int64_t)blockIdx.x * kMuThreads + inexact_cols[i];
+  const int n_in = n_inexact;
+  for (int i = 0; i < n_in; ++i) {
+    const int64_t cc = (int64_t)blockIdx.x * kMuCols + inexact_cols[i];
     if (threadIdx.x < 2 * kLimbs) limbs[threadIdx.x / kLimbs][threadIdx.x % kLimbs] = 0;
     __syncthreads();
     for (int64_t t = threadIdx.x; t < p.T; t += kMuThreads) {
@@ -296,12 +340,12 @@ __global__ void __launch_bounds__(kMuThreads) kv_mu_kernel(MuParams p) {
     }
     __syncthreads();
   }
-  if (c >= p.C) return;
+  if (warp != 0 || c >= p.C) return;
   float mu;
   if (!exact) {
     mu = 0.0f;
-    for (int i = 0; i < n_inexact; ++i)
-      if (inexact_cols[i] == (int)threadIdx.x) mu = inexact_mu[i];
+    for (int i = 0; i < n_in; ++i)
+      if (inexact_cols[i] == lane) mu = inexact_mu[i];
   } else {
     mu = (amin == 0xFFFFFFFFu) ? 0.0f : mean_from_exact_double(S, (unsigned)p.T);
   }
@@ -422,8 +466,8 @@ __global__ void __launch_bounds__(kEncThreads) kv_window_kernel(WindowParams p) 
     const float gk = g[0], gv = g[1];
     const uint2 kc = *reinterpret_cast<const uint2*>(p.base + p.off_k_codes + slot * p.slot_codes_bytes + b * 8);
     const uint2 vc = *reinterpret_cast<const uint2*>(p.base + p.off_v_codes + slot * p.slot_codes_bytes + b * 8);
-    const float ks = e4m3_to_float(p.base[p.off_k_scales + slot * p.slot_scales_bytes + b]);
-    const float vs = e4m3_to_float(p.base[p.off_v_scales + slot * p.slot_scales_bytes + b]);
+    const uint32_t ks2 = e4m3_to_f16x2_bcast(p.base[p.off_k_scales + slot * p.slot_scales_bytes + b]);
+    const uint32_t vs2 = e4m3_to_f16x2_bcast(p.base[p.off_v_scales + slot * p.slot_scales_bytes + b]);
     const float4* m4 = reinterpret_cast<const float4*>(p.base + p.off_mu + (slot * p.C + c) * 4);
     float mu[16];
 #pragma unroll
@@ -434,13 +478,21 @@ __global__ void __launch_bounds__(kEncThreads) kv_window_kernel(WindowParams p) 
       mu[4 * q + 2] = m.z;
       mu[4 * q + 3] = m.w;
     }
+    uint32_t kh[8], vh[8];
+    e2m1x8_times_scale(kc.x, ks2, *reinterpret_cast<uint32_t(*)[4]>(&kh[0]));
+    e2m1x8_times_scale(kc.y, ks2, *reinterpret_cast<uint32_t(*)[4]>(&kh[4]));
+    e2m1x8_times_scale(vc.x, vs2, *reinterpret_cast<uint32_t(*)[4]>(&vh[0]));
+    e2m1x8_times_scale(vc.y, vs2, *reinterpret_cast<uint32_t(*)[4]>(&vh[4]));
     float ko[16], vo[16];
 #pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      f16x2_to_f32x2(kh[q], ko[2 * q], ko[2 * q + 1]);  // e2m1 * s, exact
+      f16x2_to_f32x2(vh[q], vo[2 * q], vo[2 * q + 1]);
+    }
+#pragma unroll
     for (int q = 0; q < 16; ++q) {
-      const uint32_t kcode = ((q < 8 ? kc.x : kc.y) >> (4 * (q & 7))) & 0xFu;
-      const uint32_t vcode = ((q < 8 ? vc.x : vc.y) >> (4 * (q & 7))) & 0xFu;
-      ko[q] = (e2m1_to_float(kcode) * ks) * gk + mu[q];  // no fusion: -fmad=false
-      vo[q] = (e2m1_to_float(vcode) * vs) * gv;
+      ko[q] = ko[q] * gk + mu[q];  // no fusion: -fmad=false
+      vo[q] = vo[q] * gv;
     }
     uint8_t* kd = p.k_out + ob * 32;
     uint8_t* vd = p.v_out + ob * 32;
@@ -462,30 +514,35 @@ int sm_count() {
   return sms;
 }
 
-}  // namespace
-
-int64_t kv_scratch_bytes(int32_t heads, int32_t head_dim, int64_t chunk_tokens) {
-  (void)chunk_tokens;
-  const int64_t C = (int64_t)heads * head_dim;
-  return align256((int64_t)kSplits * C * 8) + 3 * align256((int64_t)kSplits * C * 4) + 256;
-}
-
-cudaError_t launch_kv_append(const KVLayout& L, const void* k, const void* v, int32_t slot,
-                             unsigned* status, cudaStream_t s) {
+// Stats -> mu -> encode for one append, statistics in `sc` (words already zeroed).
+// The token splits of the stats pass fill one wave of resident CTAs (at most
+// kSplits, the size the scratch is laid out for).
+cudaError_t launch_append_kernels(const KVLayout& L, const void* k, const void* v, int32_t slot,
+                                  const Scratch& sc, unsigned* status, cudaStream_t s) {
   const int64_t C = (int64_t)L.heads * L.head_dim;
   const int64_t T = L.chunk_tokens;
-  Scratch sc = scratch_at(L.base + L.off_scratch, C);
-  cudaError_t e = cudaMemsetAsync(sc.words, 0, 3 * sizeof(unsigned), s);
+  static int resident[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (resident[dev] == 0) {
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kv_stats_kernel, kStatsThreads, 0);
+    if (e != cudaSuccess) return e;
+    resident[dev] = max(1, per_sm) * sm_count();
+  }
+  const int64_t colblocks = (C + kStatsCols - 1) / kStatsCols;
+  const int nsplits = (int)max((int64_t)1, min((int64_t)kSplits, resident[dev] / colblocks));
 
   StatsParams sp;
   sp.k = (const uint8_t*)k;
   sp.v = (const uint8_t*)v;
   sp.T = T;
   sp.C = C;
-  sp.tokens_per_split = (T + kSplits - 1) / kSplits;
+  sp.tokens_per_split = (T + nsplits - 1) / nsplits;
   sp.sc = sc;
-  dim3 sgrid((unsigned)((C + kStatsCols - 1) / kStatsCols), kSplits);
+  dim3 sgrid((unsigned)colblocks, (unsigned)nsplits);
   kv_stats_kernel<<<sgrid, kStatsThreads, 0, s>>>(sp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
@@ -493,14 +550,14 @@ cudaError_t launch_kv_append(const KVLayout& L, const void* k, const void* v, in
   mp.k = (const uint8_t*)k;
   mp.T = T;
   mp.C = C;
+  mp.nsplits = nsplits;
   mp.sc = sc;
   mp.mu = reinterpret_cast<float*>(L.base + L.off_mu) + (int64_t)slot * C;
   int lg = 0;
   while ((1ll << lg) < T) ++lg;
   mp.log2T_ceil = lg;
-  kv_mu_kernel<<<(unsigned)((C + kMuThreads - 1) / kMuThreads), kMuThreads, 0, s>>>(mp);
+  kv_mu_kernel<<<(unsigned)((C + kMuCols - 1) / kMuCols), kMuThreads, 0, s>>>(mp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
   EncParams ep;
   ep.k = (const uint8_t*)k;
   ep.v = (const uint8_t*)v;
@@ -518,6 +575,24 @@ cudaError_t launch_kv_append(const KVLayout& L, const void* k, const void* v, in
   const int64_t cap = (int64_t)sm_count() * 8;
   kv_encode_kernel<<<(unsigned)(want < cap ? want : cap), kEncThreads, 0, s>>>(ep);
   return cudaGetLastError();
+}
+
+}  // namespace
+
+int64_t kv_scratch_bytes(int32_t heads, int32_t head_dim, int64_t chunk_tokens) {
+  (void)chunk_tokens;
+  const int64_t C = (int64_t)heads * head_dim;
+  return align256((int64_t)kSplits * C * 8) + 3 * align256((int64_t)kSplits * C * 4) + 256;
+}
+
+cudaError_t launch_kv_append(const KVLayout& L, const void* k, const void* v, int32_t slot,
+                             unsigned* status, cudaStream_t s) {
+  const int64_t C = (int64_t)L.heads * L.head_dim;
+  Scratch sc = scratch_at(L.base + L.off_scratch, C);
+  cudaError_t e = cudaMemsetAsync(sc.words, 0, 3 * sizeof(unsigned), s);
+  if (e != cudaSuccess) return e;
+
+  return launch_append_kernels(L, k, v, slot, sc, status, s);
 }
 
 cudaError_t launch_kv_window(const KVLayout& L, const int32_t* slots, int32_t n_slots, void* k_out,
@@ -584,56 +659,16 @@ static cudaError_t kv_noalloc_scratch(uint8_t** out) {
 cudaError_t launch_kv_append_noalloc(const KVLayout& L, const void* k, const void* v, int32_t slot,
                                      unsigned* status, cudaStream_t s) {
   const int64_t C = (int64_t)L.heads * L.head_dim;
-  const int64_t T = L.chunk_tokens;
   if (C > kNoAllocMaxColumns) return cudaErrorInvalidValue;
   uint8_t* scratch = nullptr;
   cudaError_t e = kv_noalloc_scratch(&scratch);
   if (e != cudaSuccess) return e;
   Scratch sc = scratch_at(scratch, C);
   // the words accumulate with atomics: they must start at zero on every call; the
-  // per-split statistics are fully rewritten by kv_stats_kernel
+  // statistics of every split in use are fully rewritten by kv_stats_kernel
   if ((e = cudaMemsetAsync(sc.words, 0, 3 * sizeof(unsigned), s)) != cudaSuccess) return e;
 
-  StatsParams sp;
-  sp.k = (const uint8_t*)k;
-  sp.v = (const uint8_t*)v;
-  sp.T = T;
-  sp.C = C;
-  sp.tokens_per_split = (T + kSplits - 1) / kSplits;
-  sp.sc = sc;
-  dim3 sgrid((unsigned)((C + kStatsCols - 1) / kStatsCols), kSplits);
-  kv_stats_kernel<<<sgrid, kStatsThreads, 0, s>>>(sp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-  MuParams mp;
-  mp.k = (const uint8_t*)k;
-  mp.T = T;
-  mp.C = C;
-  mp.sc = sc;
-  mp.mu = reinterpret_cast<float*>(L.base + L.off_mu) + (int64_t)slot * C;
-  int lg = 0;
-  while ((1ll << lg) < T) ++lg;
-  mp.log2T_ceil = lg;
-  kv_mu_kernel<<<(unsigned)((C + kMuThreads - 1) / kMuThreads), kMuThreads, 0, s>>>(mp);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
-
-  EncParams ep;
-  ep.k = (const uint8_t*)k;
-  ep.v = (const uint8_t*)v;
-  ep.nblocks = T * C / 16;
-  ep.cblocks = FastDiv((uint32_t)(C / 16));
-  ep.mu = mp.mu;
-  ep.k_codes = L.base + L.off_k_codes + (int64_t)slot * L.slot_codes_bytes;
-  ep.v_codes = L.base + L.off_v_codes + (int64_t)slot * L.slot_codes_bytes;
-  ep.k_scales = L.base + L.off_k_scales + (int64_t)slot * L.slot_scales_bytes;
-  ep.v_scales = L.base + L.off_v_scales + (int64_t)slot * L.slot_scales_bytes;
-  ep.gscale = reinterpret_cast<float*>(L.base + L.off_gscale) + 2 * (int64_t)slot;
-  ep.words = sc.words;
-  ep.status = status;
-  const int64_t want = (ep.nblocks + kEncThreads - 1) / kEncThreads;
-  const int64_t cap = (int64_t)sm_count() * 8;
-  kv_encode_kernel<<<(unsigned)(want < cap ? want : cap), kEncThreads, 0, s>>>(ep);
-  return cudaGetLastError();
+  return launch_append_kernels(L, k, v, slot, sc, status, s);
 }
 
 }  // namespace nvfp4

@@ -181,12 +181,16 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantParams p) {
     const uint32_t j = (uint32_t)b - r * p.nb_per_row.d;
     const uint2 c = *reinterpret_cast<const uint2*>(p.codes + (int64_t)r * p.ld_codes + (int64_t)j * 8);
     const int64_t soff = kMma ? sf_mma_offset(r, j, p.groups) : (int64_t)r * p.ld_scales + j;
-    const float s = e4m3_to_float(p.scales[soff]);
+    const uint32_t s2 = e4m3_to_f16x2_bcast(p.scales[soff]);
+    uint32_t h[8];
+    e2m1x8_times_scale(c.x, s2, *reinterpret_cast<uint32_t(*)[4]>(&h[0]));
+    e2m1x8_times_scale(c.y, s2, *reinterpret_cast<uint32_t(*)[4]>(&h[4]));
     float y[16];
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      const uint32_t code = ((k < 8 ? c.x : c.y) >> (4 * (k & 7))) & 0xFu;
-      y[k] = (e2m1_to_float(code) * s) * g;  // the first product is exact
+    for (int k = 0; k < 8; ++k) {
+      f16x2_to_f32x2(h[k], y[2 * k], y[2 * k + 1]);  // e2m1 * s, exact
+      y[2 * k] *= g;
+      y[2 * k + 1] *= g;
     }
     uint8_t* dst = p.y + (int64_t)r * p.y_row_bytes + (int64_t)j * (kBf16Out ? 32 : 64);
     if (kBf16Out) {
