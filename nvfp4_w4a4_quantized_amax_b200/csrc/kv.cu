@@ -409,7 +409,7 @@ __global__ void __launch_bounds__(kEncThreads) kv_encode_kernel(EncParams p) {
     const int64_t c = ((int64_t)b - (int64_t)row * p.cblocks.d) * 16;
     float kv[16], vv[16];
     {
-      const uint4 a = ldg_nc_v4(p.k + b * 32), bb = ldg_nc_v4(p.k + b * 32 + 16);
+      const uint4 a = ldg_nc_v4_l1(p.k + b * 32), bb = ldg_nc_v4_l1(p.k + b * 32 + 16);
       const uint32_t w[8] = {a.x, a.y, a.z, a.w, bb.x, bb.y, bb.z, bb.w};
       const float4* m4 = reinterpret_cast<const float4*>(p.mu + c);
       float mu[16];
@@ -428,7 +428,7 @@ __global__ void __launch_bounds__(kEncThreads) kv_encode_kernel(EncParams p) {
       }
     }
     {
-      const uint4 a = ldg_nc_v4(p.v + b * 32), bb = ldg_nc_v4(p.v + b * 32 + 16);
+      const uint4 a = ldg_nc_v4_l1(p.v + b * 32), bb = ldg_nc_v4_l1(p.v + b * 32 + 16);
       const uint32_t w[8] = {a.x, a.y, a.z, a.w, bb.x, bb.y, bb.z, bb.w};
 #pragma unroll
       for (int q = 0; q < 8; ++q) {
@@ -456,54 +456,44 @@ struct WindowParams {
 // One thread produces one 16-value block of K^ and of V^.
 __global__ void __launch_bounds__(kEncThreads) kv_window_kernel(WindowParams p) {
   const int64_t stride = (int64_t)gridDim.x * kEncThreads;
-  for (int64_t ob = (int64_t)blockIdx.x * kEncThreads + threadIdx.x; ob < p.nblocks; ob += stride) {
+  // two threads per 16-value block of K and of V (8 values each)
+  const int64_t total = 2 * p.nblocks;
+  for (int64_t oh = (int64_t)blockIdx.x * kEncThreads + threadIdx.x; oh < total; oh += stride) {
+    const int64_t ob = oh >> 1;
+    const int half = (int)(oh & 1);
     const uint32_t i = p.bpc.div((uint32_t)ob);
     const int64_t b = ob - (int64_t)i * p.blocks_per_chunk;
     const int64_t slot = p.slots[i];
     const uint32_t row = p.cblocks.div((uint32_t)b);
-    const int64_t c = (b - (int64_t)row * p.cblocks.d) * 16;
+    const int64_t c = (b - (int64_t)row * p.cblocks.d) * 16 + half * 8;
     const float* g = reinterpret_cast<const float*>(p.base + p.off_gscale) + 2 * slot;
     const float gk = g[0], gv = g[1];
-    const uint2 kc = *reinterpret_cast<const uint2*>(p.base + p.off_k_codes + slot * p.slot_codes_bytes + b * 8);
-    const uint2 vc = *reinterpret_cast<const uint2*>(p.base + p.off_v_codes + slot * p.slot_codes_bytes + b * 8);
+    const int64_t hb = 2 * b + half;
+    const uint32_t kc = *reinterpret_cast<const uint32_t*>(p.base + p.off_k_codes + slot * p.slot_codes_bytes + hb * 4);
+    const uint32_t vc = *reinterpret_cast<const uint32_t*>(p.base + p.off_v_codes + slot * p.slot_codes_bytes + hb * 4);
     const uint32_t ks2 = e4m3_to_f16x2_bcast(p.base[p.off_k_scales + slot * p.slot_scales_bytes + b]);
     const uint32_t vs2 = e4m3_to_f16x2_bcast(p.base[p.off_v_scales + slot * p.slot_scales_bytes + b]);
     const float4* m4 = reinterpret_cast<const float4*>(p.base + p.off_mu + (slot * p.C + c) * 4);
-    float mu[16];
+    const float4 m0 = m4[0], m1 = m4[1];
+    const float mu[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+    uint32_t kh[4], vh[4];
+    e2m1x8_times_scale(kc, ks2, kh);
+    e2m1x8_times_scale(vc, vs2, vh);
+    float ko[8], vo[8];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      const float4 m = m4[q];
-      mu[4 * q] = m.x;
-      mu[4 * q + 1] = m.y;
-      mu[4 * q + 2] = m.z;
-      mu[4 * q + 3] = m.w;
-    }
-    uint32_t kh[8], vh[8];
-    e2m1x8_times_scale(kc.x, ks2, *reinterpret_cast<uint32_t(*)[4]>(&kh[0]));
-    e2m1x8_times_scale(kc.y, ks2, *reinterpret_cast<uint32_t(*)[4]>(&kh[4]));
-    e2m1x8_times_scale(vc.x, vs2, *reinterpret_cast<uint32_t(*)[4]>(&vh[0]));
-    e2m1x8_times_scale(vc.y, vs2, *reinterpret_cast<uint32_t(*)[4]>(&vh[4]));
-    float ko[16], vo[16];
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
       f16x2_to_f32x2(kh[q], ko[2 * q], ko[2 * q + 1]);  // e2m1 * s, exact
       f16x2_to_f32x2(vh[q], vo[2 * q], vo[2 * q + 1]);
     }
 #pragma unroll
-    for (int q = 0; q < 16; ++q) {
+    for (int q = 0; q < 8; ++q) {
       ko[q] = ko[q] * gk + mu[q];  // no fusion: -fmad=false
       vo[q] = vo[q] * gv;
     }
-    uint8_t* kd = p.k_out + ob * 32;
-    uint8_t* vd = p.v_out + ob * 32;
-    stg_v4(kd, make_uint4(pack_bf16x2(ko[0], ko[1]), pack_bf16x2(ko[2], ko[3]),
-                          pack_bf16x2(ko[4], ko[5]), pack_bf16x2(ko[6], ko[7])));
-    stg_v4(kd + 16, make_uint4(pack_bf16x2(ko[8], ko[9]), pack_bf16x2(ko[10], ko[11]),
-                               pack_bf16x2(ko[12], ko[13]), pack_bf16x2(ko[14], ko[15])));
-    stg_v4(vd, make_uint4(pack_bf16x2(vo[0], vo[1]), pack_bf16x2(vo[2], vo[3]),
-                          pack_bf16x2(vo[4], vo[5]), pack_bf16x2(vo[6], vo[7])));
-    stg_v4(vd + 16, make_uint4(pack_bf16x2(vo[8], vo[9]), pack_bf16x2(vo[10], vo[11]),
-                               pack_bf16x2(vo[12], vo[13]), pack_bf16x2(vo[14], vo[15])));
+    stg_v4(p.k_out + oh * 16, make_uint4(pack_bf16x2(ko[0], ko[1]), pack_bf16x2(ko[2], ko[3]),
+                                         pack_bf16x2(ko[4], ko[5]), pack_bf16x2(ko[6], ko[7])));
+    stg_v4(p.v_out + oh * 16, make_uint4(pack_bf16x2(vo[0], vo[1]), pack_bf16x2(vo[2], vo[3]),
+                                         pack_bf16x2(vo[4], vo[5]), pack_bf16x2(vo[6], vo[7])));
   }
 }
 
@@ -615,7 +605,7 @@ cudaError_t launch_kv_window(const KVLayout& L, const int32_t* slots, int32_t n_
   for (int i = 0; i < kMaxWindow; ++i) p.slots[i] = i < n_slots ? slots[i] : 0;
   p.k_out = (uint8_t*)k_out;
   p.v_out = (uint8_t*)v_out;
-  const int64_t want = (p.nblocks + kEncThreads - 1) / kEncThreads;
+  const int64_t want = (2 * p.nblocks + kEncThreads - 1) / kEncThreads;
   const int64_t cap = (int64_t)sm_count() * 8;
   kv_window_kernel<<<(unsigned)(want < cap ? want : cap), kEncThreads, 0, s>>>(p);
   return cudaGetLastError();

@@ -112,7 +112,8 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(EncodeParams p) {
     float v[16];
     const uint8_t* src = p.x + (int64_t)r * p.x_row_bytes + (int64_t)j * (kBf16 ? 32 : 64);
     if (kBf16) {
-      const uint4 a = ldg_nc_v4(src), b = ldg_nc_v4(src + 16);
+      // the second load finds the other half of each 32-byte sector in L1
+      const uint4 a = ldg_nc_v4_l1(src), b = ldg_nc_v4_l1(src + 16);
       const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -122,7 +123,7 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(EncodeParams p) {
     } else {
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const uint4 a = ldg_nc_v4(src + 16 * k);
+        const uint4 a = ldg_nc_v4_l1(src + 16 * k);
         v[4 * k] = __uint_as_float(a.x);
         v[4 * k + 1] = __uint_as_float(a.y);
         v[4 * k + 2] = __uint_as_float(a.z);
@@ -171,36 +172,36 @@ struct DequantParams {
   int64_t y_row_bytes;
 };
 
-// One thread decodes one 16-value block: y = RN(RN(e2m1 * s) * g).
+// Two threads per 16-value block (8 values each): y = RN(RN(e2m1 * s) * g).  A
+// warp reads 128 contiguous bytes of codes and writes 512 contiguous bytes of bf16.
 template <bool kMma, bool kBf16Out>
 __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantParams p) {
   const float g = *p.gscale;
+  const int64_t total = 2 * p.nblocks;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < p.nblocks; b += stride) {
-    const uint32_t r = p.nb_per_row.div((uint32_t)b);
-    const uint32_t j = (uint32_t)b - r * p.nb_per_row.d;
-    const uint2 c = *reinterpret_cast<const uint2*>(p.codes + (int64_t)r * p.ld_codes + (int64_t)j * 8);
+  for (int64_t hb = (int64_t)blockIdx.x * kThreads + threadIdx.x; hb < total; hb += stride) {
+    const uint32_t b = (uint32_t)(hb >> 1);
+    const int half = (int)(hb & 1);
+    const uint32_t r = p.nb_per_row.div(b);
+    const uint32_t j = b - r * p.nb_per_row.d;
+    const uint32_t c = *reinterpret_cast<const uint32_t*>(p.codes + (int64_t)r * p.ld_codes + (int64_t)j * 8 + half * 4);
     const int64_t soff = kMma ? sf_mma_offset(r, j, p.groups) : (int64_t)r * p.ld_scales + j;
-    const uint32_t s2 = e4m3_to_f16x2_bcast(p.scales[soff]);
-    uint32_t h[8];
-    e2m1x8_times_scale(c.x, s2, *reinterpret_cast<uint32_t(*)[4]>(&h[0]));
-    e2m1x8_times_scale(c.y, s2, *reinterpret_cast<uint32_t(*)[4]>(&h[4]));
-    float y[16];
+    uint32_t h[4];
+    e2m1x8_times_scale(c, e4m3_to_f16x2_bcast(p.scales[soff]), h);
+    float y[8];
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < 4; ++k) {
       f16x2_to_f32x2(h[k], y[2 * k], y[2 * k + 1]);  // e2m1 * s, exact
       y[2 * k] *= g;
       y[2 * k + 1] *= g;
     }
-    uint8_t* dst = p.y + (int64_t)r * p.y_row_bytes + (int64_t)j * (kBf16Out ? 32 : 64);
+    uint8_t* dst = p.y + (int64_t)r * p.y_row_bytes + (int64_t)j * (kBf16Out ? 32 : 64) + half * (kBf16Out ? 16 : 32);
     if (kBf16Out) {
       stg_v4(dst, make_uint4(pack_bf16x2(y[0], y[1]), pack_bf16x2(y[2], y[3]),
                              pack_bf16x2(y[4], y[5]), pack_bf16x2(y[6], y[7])));
-      stg_v4(dst + 16, make_uint4(pack_bf16x2(y[8], y[9]), pack_bf16x2(y[10], y[11]),
-                                  pack_bf16x2(y[12], y[13]), pack_bf16x2(y[14], y[15])));
     } else {
 #pragma unroll
-      for (int k = 0; k < 4; ++k)
+      for (int k = 0; k < 2; ++k)
         stg_v4(dst + 16 * k, make_uint4(__float_as_uint(y[4 * k]), __float_as_uint(y[4 * k + 1]),
                                         __float_as_uint(y[4 * k + 2]), __float_as_uint(y[4 * k + 3])));
     }
@@ -288,7 +289,7 @@ cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t s) {
   p.nb_per_row = FastDiv((uint32_t)nb);
   p.y = (uint8_t*)a.y;
   p.y_row_bytes = a.ldy * (a.y_bf16 ? 2 : 4);
-  const int grid = grid_for(p.nblocks);
+  const int grid = grid_for(2 * p.nblocks);
   if (a.sf_mma) {
     if (a.y_bf16) dequant_kernel<true, true><<<grid, kThreads, 0, s>>>(p);
     else dequant_kernel<true, false><<<grid, kThreads, 0, s>>>(p);
