@@ -128,6 +128,23 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------- our arm
+def rank_seed_offset(rank: int) -> int:
+    """Each rank is an independent replica: its synthetic chunk uses its own seeds."""
+    return 1000 * rank
+
+
+def max_over_ranks(values, dist, device):
+    """Element-wise max of per-rank timings (the slowest rank sets the job's time);
+    identity without a process group."""
+    if dist is None:
+        return list(values)
+    import torch
+
+    t = torch.tensor(list(values), dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
 def run_ours(args, rank: int, world: int, local_rank: int):
     import torch
 
@@ -136,7 +153,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
-    seed_off = 1000 * rank
+    seed_off = rank_seed_offset(rank)
 
     def to_dev(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
@@ -304,11 +321,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         raise RuntimeError("device status: " + nv.status_string(status))
 
     # ---- max over ranks
-    ms_per_step = elapsed_ms / args.steps
-    if dist is not None:
-        t = torch.tensor([ms_per_step, e2e_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms_per_step, e2e_ms = t.tolist()
+    ms_per_step, e2e_ms = max_over_ranks([elapsed_ms / args.steps, e2e_ms], dist, dev)
     return {"ms_per_step": ms_per_step, "e2e_ms": e2e_ms, "kernels": kernels, "clocks": clocks,
             "launches": n_launch, "h2d": h2d, "d2h": d2h}
 
@@ -340,15 +353,19 @@ def summarize(res, args, world):
         ktab[name] = entry
     gemm_names = [n for n in ktab if n.startswith("gemm")]
     gemm_ms = sum(ktab[n]["ms"] for n in gemm_names)
-    achieved = flops / (gemm_ms * 1e-3) / 1e12
+    all_gemm = flops / (gemm_ms * 1e-3) / 1e12
+    # the dominant launch: the FFN-up-shaped block GEMM, 8192 x 14336 x 3072, FP32 out
+    dom = ktab["gemm_3072x14336"]
+    dom_flops = 2.0 * M_TOK * 14336 * 3072
+    achieved = dom_flops / (dom["ms"] * 1e-3) / 1e12
     step_ms = res["ms_per_step"]
     value = world * flops / (step_ms * 1e-3) / 1e12
     e2e_value = world * flops / (res["e2e_ms"] * 1e-3) / 1e12
     traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    prof = os.path.join(ROOT, "profiles", "gemm_pair_kernel_8192x14336x3072_traffic.json")
     if os.path.exists(prof):
         with open(prof) as f:
-            traffic = json.load(f).get("gemm_per_launch_bytes")
+            traffic = json.load(f).get("dram_bytes_per_launch")
     return {
         "metric": METRIC,
         "value": round(value, 2),
@@ -366,7 +383,9 @@ def summarize(res, args, world):
                    "parallelism": f"replica x{world} (independent chunks per GPU)"},
         "roofline": {"bound": "tensor", "achieved": round(achieved, 1), "peak": round(fp4_peak, 1),
                      "unit": "TFLOP/s", "frac": round(achieved / fp4_peak, 4), "traffic": traffic,
-                     "kernel": "gemm (all W4A4 GEMM launches of the step, time-weighted)",
+                     "kernel": "gemm_pair_kernel, one 8192x14336x3072 launch (FP32 out), CUDA events",
+                     "all_gemm_time_weighted": {"achieved": round(all_gemm, 1),
+                                                "frac": round(all_gemm / fp4_peak, 4)},
                      "peak_source": f"{peaks['source']} bf16 sustained x4 (dense FP4/BF16 nominal ratio)"},
         "kernels": ktab,
         "e2e": {"value": round(e2e_value, 2), "unit": "TFLOP/s", "h2d_bytes_per_step": res["h2d"],
@@ -392,13 +411,20 @@ def oracle_weights():
     return _ORACLE_WEIGHTS
 
 
-def oracle_sample_step(frac_rows: int = 128):
+def oracle_sample_step(frac_rows: int = 128, frac_cols: int = 1):
     """The oracle on a bounded sample of one step: 1/frac_rows of every row count
-    (activation rows, GEMM rows, KV tokens), weights already quantized.  Inputs
-    are generated before the clock starts.  Returns (seconds, GEMM FLOPs done)."""
+    (activation rows, GEMM rows, KV tokens) and 1/frac_cols of every GEMM's output
+    columns (a slice of the quantized weight rows), weights already quantized.
+    Inputs are generated before the clock starts.  Returns (seconds, GEMM FLOPs)."""
     import oracle
 
+    def part(q, nrows, ncols):  # a slice of a quantized tensor (indexing only)
+        return oracle.Quantized(q.codes[:nrows, : ncols // 2], q.scales[:nrows, : ncols // 16], q.g, q.amax,
+                                nrows, ncols)
+
     W = oracle_weights()
+    if frac_cols > 1:
+        W = {key: part(q, max(16, q.rows // frac_cols), q.cols) for key, q in W.items()}
     r2 = ACT_ROWS // frac_rows
     m = M_TOK // frac_rows
     t = CHUNK // frac_rows
@@ -416,16 +442,18 @@ def oracle_sample_step(frac_rows: int = 128):
     for i, (k, n) in enumerate(BLOCK_GEMMS):
         w, a = W[("blk", i)], acts[k]
         oracle.gemm_ref(a.codes, a.scales, a.g, w.codes, w.scales, w.g)
-        flops += 2.0 * m * n * k
+        flops += 2.0 * m * w.codes.shape[0] * k
     chunks = [oracle.kv_append(kk, vv) for kk, vv in kvs]
     for ch in chunks:
         oracle.kv_dequant_chunk(ch)
     qx = oracle.quantize(x5)
     c1, _ = oracle.gemm_ref(qx.codes, qx.scales, qx.g, W["w1"].codes, W["w1"].scales, W["w1"].g)
     h = oracle.gelu_tanh(c1.astype(np.float32)).astype(np.float32)
+    # the (sliced) FFN-up output feeds the first columns of FFN-down's K
+    w2 = part(W["w2"], W["w2"].rows, h.shape[1]) if frac_cols > 1 else W["w2"]
     qh = oracle.quantize(h)
-    oracle.gemm_ref(qh.codes, qh.scales, qh.g, W["w2"].codes, W["w2"].scales, W["w2"].g)
-    flops += 2 * 2.0 * m * FFN[0] * FFN[1]
+    oracle.gemm_ref(qh.codes, qh.scales, qh.g, w2.codes, w2.scales, w2.g)
+    flops += 2.0 * m * h.shape[1] * FFN[0] + 2.0 * m * w2.codes.shape[0] * h.shape[1]
     return time.perf_counter() - t0, flops
 
 
@@ -445,15 +473,15 @@ def run_reference(args, rank, world):
         return None
     oracle_weights()
     for _ in range(args.warmup):
-        oracle_sample_step(1024)
+        oracle_sample_step(1024, 16)
     secs, fl = [], 0.0
     for _ in range(args.steps):
-        s, fl = oracle_sample_step(512)
+        s, fl = oracle_sample_step(512, 16)
         secs.append(s)
     mean_s = statistics.mean(secs)
     value = fl / mean_s / 1e12
     sample = ("1/512 of every row count of one step (64 activation rows, 16 GEMM rows, 16 KV tokens "
-              "per chunk); weights quantized once before timing")
+              "per chunk) and 1/16 of every GEMM's output columns; weights quantized once before timing")
     line = {
         "impl": "reference",
         "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
