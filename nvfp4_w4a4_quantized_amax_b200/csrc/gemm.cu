@@ -699,13 +699,25 @@ struct Params2 {
   const uint8_t* sfw;
   const float* ga;
   const float* gw;
-  bool c_bf16;
+  bool has_c, c_bf16;
+  int act;
+  uint8_t* q_codes;
+  int64_t q_ld_codes;
+  uint8_t* q_scales;
+  int64_t q_groups;
+  const float* q_gscale_in;
+  float* q_gscale_out;
+  float* q_amax_out;
+  float* h_out;
   unsigned* status;
   unsigned long long wait_limit_ns;
 };
 
 // 22 warps: six share one of the SM's four 16K-register files, so at most
 // 16384 / (6 * 32) = 85 registers a thread (80 after allocation rounding).
+// kFused = false: plain FP32/bf16 output.  kFused = true: the general epilogue
+// (GELU, h_out, max|h|, NVFP4 requantization, optional C).
+template <bool kFused>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w,
                      const __grid_constant__ CUtensorMap map_c, Params2 p) {
@@ -912,12 +924,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     // Warp w reads tensor-memory lane quarter w % 4 (rows 32 (w % 4) .. + 31 of this
     // CTA's 128) and columns [64 g, 64 g + 64), g = (w - kEpiWarp0) / 4.  It takes
     // its 64 accumulator values into registers and frees the accumulator at once;
-    // the scaling and TMA stores then overlap the next tile's MMAs.
+    // the scaling, activation, requantization and stores then overlap the next
+    // tile's MMAs.
     const int quarter = warp & 3;
     const int cgroup = (warp - kEpiWarp0) / 4;
     const uint32_t leader_tempty0 = map_to_rank(smem_u32(&tempty_bar[0]), 0);
     const float gab = (*p.ga) * (*p.gw);
     const uint32_t buf = smem_u32(staging) + (uint32_t)((warp - kEpiWarp0) * kStagingBytesPerWarp);
+    float gq = 0.0f, d6q = 0.0f, r6q = 0.0f;
+    if (kFused && p.q_codes) {
+      gq = *p.q_gscale_in;
+      d6q = 6.0f * gq;
+      r6q = 1.0f / d6q;
+      if (blockIdx.x == 0 && threadIdx.x == kEpiWarp0 * 32) *p.q_gscale_out = gq;
+    }
+    const bool has_c = kFused ? p.has_c : true;
+    unsigned amax_bits = 0;
     uint32_t tcount = 0;
     for (int64_t tile = pair; tile < p.num_tiles; tile += num_pairs, ++tcount) {
       const int a = tcount % kAccStages;
@@ -937,6 +959,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive_cluster(leader_tempty0 + (uint32_t)(a * 8));
       const int64_t mt = tile % p.num_m, nt = tile / p.num_m;
       const int32_t out_row = (int32_t)(mt * kBM + rank * 128 + quarter * 32);
+      const int64_t row = (int64_t)out_row + lane;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
         const int64_t col0 = nt * kBN + cgroup * 64 + h * 32;
@@ -944,43 +967,101 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         float* v = reinterpret_cast<float*>(r[h]);
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[h][i]) * gab;
-        // the staging box is free once the previous store has read it
-        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-        __syncwarp();
-        if (p.c_bf16) {
+        if (kFused && p.act == 1) {
 #pragma unroll
-          for (int u = 0; u < 4; ++u)
-            st_shared_v4(buf + lane * 64 + ((u ^ ((lane >> 1) & 3)) * 16),
-                         make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
-                                    pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7])));
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&map_c, buf, (int32_t)col0, out_row);
-            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-          }
-        } else {
-          // FP32: two 32 x 16 boxes through the one staging box
-#pragma unroll
-          for (int b = 0; b < 2; ++b) {
-            if (b == 1) {
-              if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-              __syncwarp();
-            }
+          for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
+        }
+        if (has_c) {
+          if (p.c_bf16) {
+            // the staging box is free once the previous store has read it
+            if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+            __syncwarp();
 #pragma unroll
             for (int u = 0; u < 4; ++u)
               st_shared_v4(buf + lane * 64 + ((u ^ ((lane >> 1) & 3)) * 16),
-                           make_uint4(__float_as_uint(v[16 * b + 4 * u]), __float_as_uint(v[16 * b + 4 * u + 1]),
-                                      __float_as_uint(v[16 * b + 4 * u + 2]), __float_as_uint(v[16 * b + 4 * u + 3])));
+                           make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                                      pack_bf16x2(v[8 * u + 4], v[8 * u + 5]), pack_bf16x2(v[8 * u + 6], v[8 * u + 7])));
             asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
             __syncwarp();
             if (lane == 0) {
-              tma_store_2d(&map_c, buf, (int32_t)(col0 + 16 * b), out_row);
+              tma_store_2d(&map_c, buf, (int32_t)col0, out_row);
               asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+            }
+          } else {
+            // FP32: two 32 x 16 boxes through the one staging box
+#pragma unroll
+            for (int b = 0; b < 2; ++b) {
+              if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+              __syncwarp();
+#pragma unroll
+              for (int u = 0; u < 4; ++u)
+                st_shared_v4(buf + lane * 64 + ((u ^ ((lane >> 1) & 3)) * 16),
+                             make_uint4(__float_as_uint(v[16 * b + 4 * u]), __float_as_uint(v[16 * b + 4 * u + 1]),
+                                        __float_as_uint(v[16 * b + 4 * u + 2]), __float_as_uint(v[16 * b + 4 * u + 3])));
+              asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_2d(&map_c, buf, (int32_t)(col0 + 16 * b), out_row);
+                asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+              }
             }
           }
         }
+        if (!kFused) continue;
+        if (row >= p.M) {
+          // zero the scale padding of rows beyond M so the next GEMM reads finite scales
+          if (p.q_codes && row < (p.M + 127) / 128 * 128)
+            *reinterpret_cast<uint16_t*>(p.q_scales + sf_mma_offset(row, col0 / 16, p.q_groups)) = 0;
+          continue;
+        }
+        const int nvc = (int)min((int64_t)32, p.N - col0);  // 16 on a ragged last chunk
+        if (p.h_out) {
+          float* hd = p.h_out + row * p.N + col0;
+          if (nvc == 32) {
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              stg_v4(hd + 4 * q, make_uint4(__float_as_uint(v[4 * q]), __float_as_uint(v[4 * q + 1]),
+                                            __float_as_uint(v[4 * q + 2]), __float_as_uint(v[4 * q + 3])));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < nvc) hd[i] = v[i];
+          }
+        }
+        if (p.q_amax_out) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i)
+            if (i < nvc) amax_bits = max(amax_bits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
+        }
+        if (p.q_codes) {  // N % 64 == 0 here, so the chunk is whole
+          uint32_t w[4];
+          uint32_t sc[2];
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            float s0[8], s1[8];
+            float amax_b = 0.0f;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(v[16 * b + k]));
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+              s0[k] = v[16 * b + k];
+              s1[k] = v[16 * b + 8 + k];
+            }
+            const uint32_t s = block_scale_fast(amax_b, d6q, r6q);
+            const BlockEncoder enc(e4m3_to_float(s) * gq);
+            w[2 * b] = enc.encode8s(s0);
+            w[2 * b + 1] = enc.encode8s(s1);
+            sc[b] = s;
+          }
+          stg_v4(p.q_codes + row * p.q_ld_codes + col0 / 2, make_uint4(w[0], w[1], w[2], w[3]));
+          *reinterpret_cast<uint16_t*>(p.q_scales + sf_mma_offset(row, col0 / 16, p.q_groups)) =
+              (uint16_t)(sc[0] | (sc[1] << 8));
+        }
       }
+    }
+    if (kFused && p.q_amax_out) {
+      amax_bits = warp_max_u32(amax_bits);
+      if (lane == 0 && amax_bits) atomicMax(reinterpret_cast<unsigned*>(p.q_amax_out), amax_bits);
     }
     if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
     __syncwarp();
@@ -1073,6 +1154,7 @@ int sm_count_gemm() {
   return sms;
 }
 
+template <bool kFused>
 cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s) {
   pair::Params2 p;
   p.M = g.M;
@@ -1089,16 +1171,31 @@ cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s) {
   p.sfw = g.w.scales;
   p.ga = g.a.gscale;
   p.gw = g.w.gscale;
+  p.has_c = g.c != nullptr;
   p.c_bf16 = g.c_bf16;
+  p.act = g.act;
+  p.q_codes = g.q_codes;
+  p.q_ld_codes = g.q_ld_codes;
+  p.q_scales = g.q_scales;
+  p.q_groups = (g.N / 16 + 3) / 4;
+  p.q_gscale_in = g.q_gscale_in;
+  p.q_gscale_out = g.q_gscale_out;
+  p.q_amax_out = g.q_amax_out;
+  p.h_out = g.h_out;
   p.status = g.status;
   p.wait_limit_ns = kWaitLimitNs;
 
   CUtensorMap ma, mw, mc;
   if (!make_code_map(&ma, g.a.codes, g.M, g.K / 2, g.a.ld_codes, 128)) return cudaErrorInvalidValue;
   if (!make_code_map(&mw, g.w.codes, g.N, g.K / 2, g.w.ld_codes, pair::kBNHalf)) return cudaErrorInvalidValue;
-  if (!make_out_map(&mc, g.c, g.M, g.N, g.ldc, g.c_bf16, true)) return cudaErrorInvalidValue;
+  memset(&mc, 0, sizeof(mc));
+  if (g.c && !make_out_map(&mc, g.c, g.M, g.N, g.ldc, g.c_bf16, true)) return cudaErrorInvalidValue;
+  if (g.q_amax_out) {
+    cudaError_t e = cudaMemsetAsync(g.q_amax_out, 0, sizeof(float), s);
+    if (e != cudaSuccess) return e;
+  }
   static bool done[64];
-  cudaError_t e = set_smem_once(pair::gemm_pair_kernel, pair::kSmemBytes, done);
+  cudaError_t e = set_smem_once(pair::gemm_pair_kernel<kFused>, pair::kSmemBytes, done);
   if (e != cudaSuccess) return e;
   // Pairs must fit inside one GPC, so fewer than SMs / 2 of them may be resident
   // at once; a persistent grid larger than that would run a second wave.
@@ -1121,26 +1218,26 @@ cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s) {
     cfg.attrs = &attr;
     cfg.numAttrs = 1;
     int n = 0;
-    e = cudaOccupancyMaxActiveClusters(&n, pair::gemm_pair_kernel, &cfg);
+    e = cudaOccupancyMaxActiveClusters(&n, pair::gemm_pair_kernel<kFused>, &cfg);
     if (e != cudaSuccess) return e;
     if (n <= 0) return cudaErrorInvalidConfiguration;
     resident[dev] = n;
   }
   const int64_t max_pairs = resident[dev];
   const int64_t pairs = p.num_tiles < max_pairs ? p.num_tiles : max_pairs;
-  pair::gemm_pair_kernel<<<(unsigned)(2 * pairs), pair::kThreads, pair::kSmemBytes, s>>>(ma, mw, mc, p);
+  pair::gemm_pair_kernel<kFused><<<(unsigned)(2 * pairs), pair::kThreads, pair::kSmemBytes, s>>>(ma, mw, mc, p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
   if (g.M == 0 || g.N == 0) return cudaSuccess;
-  // Plain C output with at least one full pair tile of rows and columns: the
-  // CTA-pair kernel (256 x 256 tiles, one accumulator stage).  The fused GELU /
-  // requantization epilogue and small shapes: the single-CTA kernel, whose two
-  // accumulator stages overlap its heavier epilogue with the next tile's MMAs.
+  // At least one full pair tile of rows and columns: the CTA-pair kernel (256 x 256
+  // tiles), its plain-output instance or the one with the general epilogue.  Smaller
+  // shapes: the single-CTA kernel (128 x 128 tiles).
   const bool plain = g.c != nullptr && g.act == 0 && g.q_codes == nullptr && g.h_out == nullptr &&
                      g.q_amax_out == nullptr;
-  if (plain && g.M >= pair::kBM && g.N >= pair::kBN) return launch_gemm_pair(g, s);
+  if (g.M >= pair::kBM && g.N >= pair::kBN)
+    return plain ? launch_gemm_pair<false>(g, s) : launch_gemm_pair<true>(g, s);
   Params p;
   p.M = g.M;
   p.N = g.N;
