@@ -101,7 +101,10 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(EncodeParams p) {
 
   unsigned local_max = 0;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
-  for (int64_t vb = (int64_t)blockIdx.x * kThreads + threadIdx.x; vb < p.nvblocks; vb += stride) {
+  // Blocks are visited from the end of x backwards: the amax pass read x front to
+  // back, so its most recent reads (still in L2) are encoded first.
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < p.nvblocks; i += stride) {
+    const int64_t vb = p.nvblocks - 1 - i;
     const uint32_t r = p.vb_per_row.div((uint32_t)vb);
     const uint32_t j = (uint32_t)vb - r * p.vb_per_row.d;
     const int64_t soff = kMma ? sf_mma_offset(r, j, p.groups) : (int64_t)r * p.ld_scales + j;
