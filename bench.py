@@ -543,6 +543,19 @@ def run_single_kernel(args):
         y = torch.empty((R, C), dtype=torch.bfloat16, device=dev)
         fn = (lambda: nv.nvfp4_quantize(x, q, amax_out=amax[0:1])) if args.kernel == "quantize" else \
             (lambda: nv.nvfp4_dequantize(q, y))
+    elif args.kernel == "kv_window_sink":
+        # sink-aware window: a 1024-token sink slot, a 4096-token shot-sink slot, three
+        # full sliding slots and the newest, partial slot (3000 tokens): 32696 tokens
+        off = synth.kv_offsets(3, HEADS, HEAD_DIM)
+        k, v = synth.kv_chunk(3, 0, CHUNK, HEADS, HEAD_DIM, off)
+        kd, vd = to_dev(k), to_dev(v)
+        cache = nv.KVCache(HEADS, HEAD_DIM, CHUNK, 6, dev)
+        fills = [1024, 4096, CHUNK, CHUNK, CHUNK, 3000]
+        for sl, n in enumerate(fills):
+            nv.kv_quant_append(cache, kd[:n], vd[:n], sl)
+        ko = torch.empty((sum(fills), HEADS, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+        vo = torch.empty_like(ko)
+        fn = lambda: nv.kv_dequant_window_tokens(cache, list(range(6)), fills, ko, vo)  # noqa: E731
     elif args.kernel in ("kv_append", "kv_window"):
         off = synth.kv_offsets(3, HEADS, HEAD_DIM)
         k, v = synth.kv_chunk(3, 0, CHUNK, HEADS, HEAD_DIM, off)
@@ -580,7 +593,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel", default=None,
-                    help="profiling mode: gemm | gemm_fused | quantize | dequantize | kv_append | kv_window")
+                    help="profiling mode: gemm | gemm_fused | quantize | dequantize | kv_append | kv_window | kv_window_sink")
     ap.add_argument("--shape", default="8192,14336,3072", help="M,N,K for gemm; rows,cols for (de)quantize")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--kernel-warmup", type=int, default=1,

@@ -180,7 +180,10 @@ nvfp4_status nvfp4_gemm(const nvfp4_tensor* A, const nvfp4_tensor* W, void* C, i
  *   k_scales[max_chunks][chunk_tokens][heads][head_dim/16]  (same for v_scales)
  *   mu      [max_chunks][heads][head_dim] FP32
  *   gscale  [max_chunks][2] FP32 (g_K, g_V)
+ *   tokens  [max_chunks] int32: tokens held by each slot (written by every append)
  *   scratch used by kv_quant_append (per-column statistics of one chunk).
+ * A slot may hold fewer tokens than chunk_tokens (a partial chunk, e.g. the last
+ * chunk of a sequence or a sink chunk); its tokens are the first ones of the slot.
  */
 typedef struct nvfp4_kv_cache {
   uint8_t* base;          /* device allocation given to nvfp4_kv_cache_init */
@@ -191,7 +194,7 @@ typedef struct nvfp4_kv_cache {
   int32_t max_chunks;
   int32_t reserved;
   int64_t off_k_codes, off_v_codes, off_k_scales, off_v_scales;
-  int64_t off_mu, off_gscale, off_scratch;
+  int64_t off_mu, off_gscale, off_tokens, off_scratch;
   int64_t slot_codes_bytes;   /* chunk_tokens * heads * head_dim / 2  */
   int64_t slot_scales_bytes;  /* chunk_tokens * heads * head_dim / 16 */
 } nvfp4_kv_cache;
@@ -208,7 +211,8 @@ nvfp4_status nvfp4_kv_cache_init(void* dev_mem, size_t bytes, int32_t heads, int
 
 /* kv_quant_append — quantize one chunk of K and V into slot `slot`, in place.
  *   k, v   : device bf16 [tokens][heads][head_dim], 16-byte aligned.
- *   tokens : must equal cache->chunk_tokens.
+ *   tokens : 1 .. cache->chunk_tokens; the mean mu is over these tokens and the
+ *            slot records the count (a partial chunk holds its tokens first).
  * Appends to one cache must be issued on one stream (they share the scratch).
  * Device status NONFINITE on NaN/Inf input (the slot is then left unchanged). */
 nvfp4_status kv_quant_append(const nvfp4_kv_cache* cache, const void* k, const void* v,
@@ -243,10 +247,27 @@ nvfp4_status kv_quant_append_noalloc(const nvfp4_kv_cache* cache, const void* k,
  * of n_slots slot ids, 1 <= n_slots <= 64, repeats allowed, any order) in one
  * launch, writing bf16 [n_slots * chunk_tokens][heads][head_dim] to k_out and
  * v_out (device, 16-byte aligned) in list order:
- *   K^ = bf16(RN(RN(RN(e2m1 * s) * g_K) + mu)),  V^ = bf16(RN(RN(e2m1 * s) * g_V)). */
+ *   K^ = bf16(RN(RN(RN(e2m1 * s) * g_K) + mu)),  V^ = bf16(RN(RN(e2m1 * s) * g_V)).
+ * Every listed slot must hold chunk_tokens tokens: a slot recorded with another
+ * count sets device status NVFP4_ERR_SHAPE and its part of the output is not
+ * written. */
 nvfp4_status kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t* slots_host,
                                int32_t n_slots, void* k_out, void* v_out,
                                nvfp4_stream_t stream);
+
+/* kv_dequant_window_tokens — the same window over slots holding any number of
+ * tokens, e.g. a sink-aware window: a sink slot, some shot-sink slots and the
+ * sliding slots, possibly partial.  [TW] §四: one parallel kernel dequantizes the
+ * window's chunks together.
+ *   tokens_host : HOST array, tokens_host[i] = tokens held by slots_host[i]
+ *                 (1 .. chunk_tokens).
+ * Output: bf16 [sum(tokens_host)][heads][head_dim], the slots' tokens one after
+ * the other in list order.  A slot whose recorded count differs from the stated
+ * one sets device status NVFP4_ERR_SHAPE and its part of the output is not
+ * written. */
+nvfp4_status kv_dequant_window_tokens(const nvfp4_kv_cache* cache, const int32_t* slots_host,
+                                      const int32_t* tokens_host, int32_t n_slots, void* k_out,
+                                      void* v_out, nvfp4_stream_t stream);
 
 /* ----------------------------------------------------------------- status ----
  * Reads the sticky device status word of CUDA device `device` (synchronizes that

@@ -56,13 +56,14 @@ class nvfp4_kv_cache(ctypes.Structure):
                 ("off_k_codes", ctypes.c_int64), ("off_v_codes", ctypes.c_int64),
                 ("off_k_scales", ctypes.c_int64), ("off_v_scales", ctypes.c_int64),
                 ("off_mu", ctypes.c_int64), ("off_gscale", ctypes.c_int64),
-                ("off_scratch", ctypes.c_int64), ("slot_codes_bytes", ctypes.c_int64),
+                ("off_tokens", ctypes.c_int64), ("off_scratch", ctypes.c_int64),
+                ("slot_codes_bytes", ctypes.c_int64),
                 ("slot_scales_bytes", ctypes.c_int64)]
 
 
 EXPORTS = ["nvfp4_version", "nvfp4_status_string", "nvfp4_scales_bytes", "nvfp4_quantize",
            "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_cache_bytes", "nvfp4_kv_cache_init",
-           "kv_quant_append", "kv_quant_append_noalloc", "kv_dequant_window",
+           "kv_quant_append", "kv_quant_append_noalloc", "kv_dequant_window", "kv_dequant_window_tokens",
            "nvfp4_get_device_status"]
 
 
@@ -99,6 +100,9 @@ def library():
             lib.kv_quant_append_noalloc.argtypes = [KV, vp, vp, i64, i32, vp]
             lib.kv_dequant_window.restype = i32
             lib.kv_dequant_window.argtypes = [KV, ctypes.POINTER(ctypes.c_int32), i32, vp, vp, vp]
+            lib.kv_dequant_window_tokens.restype = i32
+            lib.kv_dequant_window_tokens.argtypes = [KV, ctypes.POINTER(ctypes.c_int32),
+                                                     ctypes.POINTER(ctypes.c_int32), i32, vp, vp, vp]
             lib.nvfp4_get_device_status.restype = i32
             lib.nvfp4_get_device_status.argtypes = [i32, ctypes.POINTER(ctypes.c_int32), i32]
             _lib = lib
@@ -238,9 +242,16 @@ class KVCache:
         g = self._view(h.off_gscale + slot * 8, 8).view(torch.float32)
         return kc, ks, vc, vs, mu, g
 
+    def slot_tokens(self, slot: int) -> int:
+        """Tokens recorded for `slot` by its last append (reads the device)."""
+        import torch
+
+        return int(self._view(self.handle.off_tokens + slot * 4, 4).view(torch.int32).item())
+
 
 def kv_quant_append(cache: KVCache, k, v, slot: int, stream=None):
-    """Quantize one chunk (bf16 [tokens, heads, head_dim]) of K and V into `slot`."""
+    """Quantize one chunk (bf16 [tokens, heads, head_dim], 1 <= tokens <= chunk_tokens)
+    of K and V into `slot`."""
     _check(library().kv_quant_append(ctypes.byref(cache.handle), _ptr(k), _ptr(v), k.shape[0], slot,
                                      _stream(stream)), "kv_quant_append")
 
@@ -258,6 +269,17 @@ def kv_dequant_window(cache: KVCache, slots: Sequence[int], k_out, v_out, stream
     arr = (ctypes.c_int32 * len(slots))(*slots)
     _check(library().kv_dequant_window(ctypes.byref(cache.handle), arr, len(slots), _ptr(k_out),
                                        _ptr(v_out), _stream(stream)), "kv_dequant_window")
+
+
+def kv_dequant_window_tokens(cache: KVCache, slots: Sequence[int], tokens: Sequence[int], k_out, v_out,
+                             stream=None):
+    """Window over slots holding tokens[i] tokens each; output rows sum(tokens), in list order."""
+    if len(tokens) != len(slots):
+        raise ValueError("one token count per slot")
+    sarr = (ctypes.c_int32 * len(slots))(*slots)
+    tarr = (ctypes.c_int32 * len(tokens))(*tokens)
+    _check(library().kv_dequant_window_tokens(ctypes.byref(cache.handle), sarr, tarr, len(slots), _ptr(k_out),
+                                              _ptr(v_out), _stream(stream)), "kv_dequant_window_tokens")
 
 
 def get_device_status(device: int = 0, clear: bool = False) -> int:

@@ -241,6 +241,7 @@ static nvfp4_status kv_geometry(int32_t heads, int32_t head_dim, int64_t chunk_t
   L->off_v_scales = o; o += align256(scales * max_chunks);
   L->off_mu = o;       o += align256(C * 4 * (int64_t)max_chunks);
   L->off_gscale = o;   o += align256(8 * (int64_t)max_chunks);
+  L->off_tokens = o;   o += align256(4 * (int64_t)max_chunks);
   L->off_scratch = o;  o += align256(nvfp4::kv_scratch_bytes(heads, head_dim, chunk_tokens));
   *total = (size_t)o;
   return NVFP4_OK;
@@ -275,6 +276,7 @@ nvfp4_status nvfp4_kv_cache_init(void* dev_mem, size_t bytes, int32_t heads, int
   cache->off_v_scales = L.off_v_scales;
   cache->off_mu = L.off_mu;
   cache->off_gscale = L.off_gscale;
+  cache->off_tokens = L.off_tokens;
   cache->off_scratch = L.off_scratch;
   cache->slot_codes_bytes = L.slot_codes_bytes;
   cache->slot_scales_bytes = L.slot_scales_bytes;
@@ -287,7 +289,8 @@ static nvfp4_status check_cache(const nvfp4_kv_cache* c, nvfp4::KVLayout* L) {
   size_t need = 0;
   nvfp4_status st = kv_geometry(c->heads, c->head_dim, c->chunk_tokens, c->max_chunks, L, &need);
   if (st != NVFP4_OK) return st;
-  if (c->bytes < need || L->off_scratch != c->off_scratch || L->off_mu != c->off_mu)
+  if (c->bytes < need || L->off_scratch != c->off_scratch || L->off_mu != c->off_mu ||
+      L->off_tokens != c->off_tokens)
     return NVFP4_ERR_INVALID_ARG;
   L->base = c->base;
   return NVFP4_OK;
@@ -300,11 +303,11 @@ nvfp4_status kv_quant_append(const nvfp4_kv_cache* cache, const void* k, const v
   if (st != NVFP4_OK) return st;
   if (!k || !v) return NVFP4_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v)) return NVFP4_ERR_ALIGNMENT;
-  if (tokens != cache->chunk_tokens) return NVFP4_ERR_SHAPE;
+  if (tokens < 1 || tokens > cache->chunk_tokens) return NVFP4_ERR_SHAPE;
   if (slot < 0 || slot >= cache->max_chunks) return NVFP4_ERR_INVALID_ARG;
   unsigned* status = nullptr;
   if ((st = current_device(&status)) != NVFP4_OK) return st;
-  return cuda_status(nvfp4::launch_kv_append(L, k, v, slot, status,
+  return cuda_status(nvfp4::launch_kv_append(L, k, v, tokens, slot, status,
                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -315,31 +318,45 @@ nvfp4_status kv_quant_append_noalloc(const nvfp4_kv_cache* cache, const void* k,
   if (st != NVFP4_OK) return st;
   if (!k || !v) return NVFP4_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v)) return NVFP4_ERR_ALIGNMENT;
-  if (tokens != cache->chunk_tokens) return NVFP4_ERR_SHAPE;
+  if (tokens < 1 || tokens > cache->chunk_tokens) return NVFP4_ERR_SHAPE;
   if (slot < 0 || slot >= cache->max_chunks) return NVFP4_ERR_INVALID_ARG;
   if ((int64_t)cache->heads * cache->head_dim > NVFP4_NOALLOC_MAX_COLUMNS) return NVFP4_ERR_SHAPE;
   unsigned* status = nullptr;
   if ((st = current_device(&status)) != NVFP4_OK) return st;
-  return cuda_status(nvfp4::launch_kv_append_noalloc(L, k, v, slot, status,
+  return cuda_status(nvfp4::launch_kv_append_noalloc(L, k, v, tokens, slot, status,
                                                      reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status kv_dequant_window_tokens(const nvfp4_kv_cache* cache, const int32_t* slots_host,
+                                      const int32_t* tokens_host, int32_t n_slots, void* k_out,
+                                      void* v_out, nvfp4_stream_t stream) {
+  nvfp4::KVLayout L;
+  nvfp4_status st = check_cache(cache, &L);
+  if (st != NVFP4_OK) return st;
+  if (!slots_host || !tokens_host || !k_out || !v_out) return NVFP4_ERR_INVALID_ARG;
+  if (n_slots < 1 || n_slots > nvfp4::kMaxWindowSlots) return NVFP4_ERR_INVALID_ARG;
+  int64_t total = 0;
+  for (int i = 0; i < n_slots; ++i) {
+    if (slots_host[i] < 0 || slots_host[i] >= cache->max_chunks) return NVFP4_ERR_INVALID_ARG;
+    if (tokens_host[i] < 1 || tokens_host[i] > cache->chunk_tokens) return NVFP4_ERR_SHAPE;
+    total += tokens_host[i];
+  }
+  if (!aligned16(k_out) || !aligned16(v_out)) return NVFP4_ERR_ALIGNMENT;
+  const int64_t C = (int64_t)cache->heads * cache->head_dim;
+  if (total * C / 16 >= kMaxBlocks) return NVFP4_ERR_SHAPE;
+  unsigned* status = nullptr;
+  if ((st = current_device(&status)) != NVFP4_OK) return st;
+  return cuda_status(nvfp4::launch_kv_window(L, slots_host, tokens_host, n_slots, k_out, v_out, status,
+                                             reinterpret_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t* slots_host,
                                int32_t n_slots, void* k_out, void* v_out, nvfp4_stream_t stream) {
-  nvfp4::KVLayout L;
-  nvfp4_status st = check_cache(cache, &L);
-  if (st != NVFP4_OK) return st;
-  if (!slots_host || !k_out || !v_out) return NVFP4_ERR_INVALID_ARG;
-  if (n_slots < 1 || n_slots > 64) return NVFP4_ERR_INVALID_ARG;
-  for (int i = 0; i < n_slots; ++i)
-    if (slots_host[i] < 0 || slots_host[i] >= cache->max_chunks) return NVFP4_ERR_INVALID_ARG;
-  if (!aligned16(k_out) || !aligned16(v_out)) return NVFP4_ERR_ALIGNMENT;
-  const int64_t C = (int64_t)cache->heads * cache->head_dim;
-  if ((int64_t)n_slots * cache->chunk_tokens * C / 16 >= kMaxBlocks) return NVFP4_ERR_SHAPE;
-  unsigned* status = nullptr;
-  if ((st = current_device(&status)) != NVFP4_OK) return st;
-  return cuda_status(nvfp4::launch_kv_window(L, slots_host, n_slots, k_out, v_out,
-                                             reinterpret_cast<cudaStream_t>(stream)));
+  if (!cache || n_slots < 1 || n_slots > nvfp4::kMaxWindowSlots) return NVFP4_ERR_INVALID_ARG;
+  if (cache->chunk_tokens > (1 << 24)) return NVFP4_ERR_SHAPE;
+  int32_t tokens[nvfp4::kMaxWindowSlots];
+  for (int i = 0; i < n_slots; ++i) tokens[i] = (int32_t)cache->chunk_tokens;
+  return kv_dequant_window_tokens(cache, slots_host, tokens, n_slots, k_out, v_out, stream);
 }
 
 nvfp4_status nvfp4_get_device_status(int32_t device, int32_t* status_out, int32_t clear) {

@@ -17,7 +17,7 @@
 
 namespace nvfp4 {
 
-enum : unsigned { kStatusOk = 0, kStatusNonfinite = 4, kStatusTimeout = 5 };
+enum : unsigned { kStatusOk = 0, kStatusShape = 2, kStatusNonfinite = 4, kStatusTimeout = 5 };
 
 // The first data error wins; later ones leave the word unchanged (sticky).
 __device__ __forceinline__ void set_status(unsigned* status, unsigned code) {

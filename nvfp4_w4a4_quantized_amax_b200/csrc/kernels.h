@@ -8,6 +8,31 @@
 
 namespace nvfp4 {
 
+// CTAs of `kThreads` threads of kernel K that are resident at once on the current
+// device (occupancy x SMs), looked up once per device: grid-stride kernels launch
+// exactly one full wave.
+template <auto K>
+int resident_ctas(int threads) {
+  static int cache[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cache[dev] == 0) {
+    int per_sm = 0, sms = 148;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, K, threads, 0) != cudaSuccess) per_sm = 1;
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = (per_sm > 0 ? per_sm : 1) * sms;
+  }
+  return cache[dev];
+}
+
+// One wave of K, or fewer CTAs when `work` items (one per thread) need fewer.
+template <auto K>
+int wave_grid(int threads, int64_t work) {
+  const int64_t want = (work + threads - 1) / threads;
+  const int64_t cap = resident_ctas<K>(threads);
+  return (int)(want < cap ? (want > 0 ? want : 1) : cap);
+}
+
 struct QuantizeArgs {
   const void* x;
   bool x_bf16;
@@ -43,19 +68,23 @@ struct KVLayout {
   int32_t heads, head_dim;
   int64_t chunk_tokens;
   int32_t max_chunks;
-  int64_t off_k_codes, off_v_codes, off_k_scales, off_v_scales, off_mu, off_gscale, off_scratch;
+  int64_t off_k_codes, off_v_codes, off_k_scales, off_v_scales, off_mu, off_gscale, off_tokens, off_scratch;
   int64_t slot_codes_bytes, slot_scales_bytes;
 };
 int64_t kv_scratch_bytes(int32_t heads, int32_t head_dim, int64_t chunk_tokens);
-cudaError_t launch_kv_append(const KVLayout& c, const void* k, const void* v, int32_t slot,
+// tokens: 1 .. chunk_tokens (a partial chunk fills the first tokens of the slot)
+cudaError_t launch_kv_append(const KVLayout& c, const void* k, const void* v, int64_t tokens, int32_t slot,
                              unsigned* status, cudaStream_t s);
 // Same append, but the statistics scratch is a static device array of the library
 // (at most kNoAllocMaxColumns columns) instead of the cache's scratch region.
 constexpr int64_t kNoAllocMaxColumns = 4096;
-cudaError_t launch_kv_append_noalloc(const KVLayout& c, const void* k, const void* v, int32_t slot,
-                                     unsigned* status, cudaStream_t s);
-cudaError_t launch_kv_window(const KVLayout& c, const int32_t* slots, int32_t n_slots, void* k_out,
-                             void* v_out, cudaStream_t s);
+cudaError_t launch_kv_append_noalloc(const KVLayout& c, const void* k, const void* v, int64_t tokens,
+                                     int32_t slot, unsigned* status, cudaStream_t s);
+// tokens[i]: tokens held by slots[i] (checked on the device against the slot's
+// recorded count); the output packs the slots' tokens in list order.
+constexpr int kMaxWindowSlots = 64;
+cudaError_t launch_kv_window(const KVLayout& c, const int32_t* slots, const int32_t* tokens, int32_t n_slots,
+                             void* k_out, void* v_out, unsigned* status, cudaStream_t s);
 
 struct GemmOperand {
   const uint8_t* codes;

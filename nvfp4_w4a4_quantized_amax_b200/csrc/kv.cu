@@ -35,7 +35,6 @@ constexpr int kStatsUnroll = 4;      // token rows in flight per warp
 constexpr int kMuThreads = 256;      // 8 warps share the splits of kMuCols columns
 constexpr int kMuCols = 32;
 constexpr int kEncThreads = 256;
-constexpr int kMaxWindow = 64;
 
 // scratch layout (byte offsets from the scratch base)
 struct Scratch {
@@ -366,6 +365,8 @@ struct EncParams {
   uint8_t* k_scales;
   uint8_t* v_scales;
   float* gscale;      // slot's (g_K, g_V)
+  int32_t* slot_tokens;  // slot's recorded token count
+  int32_t tokens;
   const unsigned* words;
   unsigned* status;
 };
@@ -400,6 +401,7 @@ __global__ void __launch_bounds__(kEncThreads) kv_encode_kernel(EncParams p) {
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     p.gscale[0] = gk;
     p.gscale[1] = gv;
+    *p.slot_tokens = p.tokens;
   }
   const float d6k = 6.0f * gk, d6v = 6.0f * gv;
   const float r6k = 1.0f / d6k, r6v = 1.0f / d6v;
@@ -443,36 +445,52 @@ __global__ void __launch_bounds__(kEncThreads) kv_encode_kernel(EncParams p) {
 
 struct WindowParams {
   const uint8_t* base;
-  int64_t off_k_codes, off_v_codes, off_k_scales, off_v_scales, off_mu, off_gscale;
+  int64_t off_k_codes, off_v_codes, off_k_scales, off_v_scales, off_mu, off_gscale, off_tokens;
   int64_t slot_codes_bytes, slot_scales_bytes, C;
-  int64_t blocks_per_chunk;  // T * C / 16
-  FastDiv bpc, cblocks;
-  int64_t nblocks;           // n_slots * blocks_per_chunk
-  int32_t slots[kMaxWindow];
+  FastDiv cblocks;           // C / 16
+  int32_t n_slots;
+  int32_t slots[kMaxWindowSlots];
+  int32_t tokens[kMaxWindowSlots];
+  int64_t hb_end[kMaxWindowSlots];  // cumulative half-blocks (8 values) through list entry i
   uint8_t* k_out;
   uint8_t* v_out;
+  unsigned* status;
 };
 
-// One thread produces one 16-value block of K^ and of V^.
+// One flat sweep over the output (the listed slots' tokens one after the other),
+// two threads per 16-value block of K and of V (8 values each): half-block hb of
+// the output is written at byte 16 hb of k_out / v_out.  A thread tracks the list
+// entry its index falls in and moves on as its index advances.
 __global__ void __launch_bounds__(kEncThreads) kv_window_kernel(WindowParams p) {
+  const int64_t total = p.hb_end[p.n_slots - 1];
   const int64_t stride = (int64_t)gridDim.x * kEncThreads;
-  // two threads per 16-value block of K and of V (8 values each)
-  const int64_t total = 2 * p.nblocks;
-  for (int64_t oh = (int64_t)blockIdx.x * kEncThreads + threadIdx.x; oh < total; oh += stride) {
-    const int64_t ob = oh >> 1;
-    const int half = (int)(oh & 1);
-    const uint32_t i = p.bpc.div((uint32_t)ob);
-    const int64_t b = ob - (int64_t)i * p.blocks_per_chunk;
-    const int64_t slot = p.slots[i];
+  int i = -1;
+  int64_t begin = 0, end = 0, slot = 0;
+  bool ok = false;
+  float gk = 0.0f, gv = 0.0f;
+  for (int64_t hb = (int64_t)blockIdx.x * kEncThreads + threadIdx.x; hb < total; hb += stride) {
+    while (hb >= end) {  // next list entry (a stride may skip short ones)
+      ++i;
+      begin = end;
+      end = p.hb_end[i];
+      slot = p.slots[i];
+      ok = reinterpret_cast<const int32_t*>(p.base + p.off_tokens)[slot] == p.tokens[i];
+      if (!ok && hb == begin) set_status(p.status, kStatusShape);
+      const float* g = reinterpret_cast<const float*>(p.base + p.off_gscale) + 2 * slot;
+      gk = g[0];
+      gv = g[1];
+    }
+    if (!ok) continue;
+    const int64_t lh = hb - begin;  // half-block within the slot
+    const int64_t b = lh >> 1;
+    const int half = (int)(lh & 1);
     const uint32_t row = p.cblocks.div((uint32_t)b);
     const int64_t c = (b - (int64_t)row * p.cblocks.d) * 16 + half * 8;
-    const float* g = reinterpret_cast<const float*>(p.base + p.off_gscale) + 2 * slot;
-    const float gk = g[0], gv = g[1];
-    const int64_t hb = 2 * b + half;
-    const uint32_t kc = *reinterpret_cast<const uint32_t*>(p.base + p.off_k_codes + slot * p.slot_codes_bytes + hb * 4);
-    const uint32_t vc = *reinterpret_cast<const uint32_t*>(p.base + p.off_v_codes + slot * p.slot_codes_bytes + hb * 4);
-    const uint32_t ks2 = e4m3_to_f16x2_bcast(p.base[p.off_k_scales + slot * p.slot_scales_bytes + b]);
-    const uint32_t vs2 = e4m3_to_f16x2_bcast(p.base[p.off_v_scales + slot * p.slot_scales_bytes + b]);
+    const int64_t cofs = slot * p.slot_codes_bytes + lh * 4, sofs = slot * p.slot_scales_bytes + b;
+    const uint32_t kc = *reinterpret_cast<const uint32_t*>(p.base + p.off_k_codes + cofs);
+    const uint32_t vc = *reinterpret_cast<const uint32_t*>(p.base + p.off_v_codes + cofs);
+    const uint32_t ks2 = e4m3_to_f16x2_bcast(p.base[p.off_k_scales + sofs]);
+    const uint32_t vs2 = e4m3_to_f16x2_bcast(p.base[p.off_v_scales + sofs]);
     const float4* m4 = reinterpret_cast<const float4*>(p.base + p.off_mu + (slot * p.C + c) * 4);
     const float4 m0 = m4[0], m1 = m4[1];
     const float mu[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
@@ -490,9 +508,9 @@ __global__ void __launch_bounds__(kEncThreads) kv_window_kernel(WindowParams p) 
       ko[q] = ko[q] * gk + mu[q];  // no fusion: -fmad=false
       vo[q] = vo[q] * gv;
     }
-    stg_v4(p.k_out + oh * 16, make_uint4(pack_bf16x2(ko[0], ko[1]), pack_bf16x2(ko[2], ko[3]),
+    stg_v4(p.k_out + hb * 16, make_uint4(pack_bf16x2(ko[0], ko[1]), pack_bf16x2(ko[2], ko[3]),
                                          pack_bf16x2(ko[4], ko[5]), pack_bf16x2(ko[6], ko[7])));
-    stg_v4(p.v_out + oh * 16, make_uint4(pack_bf16x2(vo[0], vo[1]), pack_bf16x2(vo[2], vo[3]),
+    stg_v4(p.v_out + hb * 16, make_uint4(pack_bf16x2(vo[0], vo[1]), pack_bf16x2(vo[2], vo[3]),
                                          pack_bf16x2(vo[4], vo[5]), pack_bf16x2(vo[6], vo[7])));
   }
 }
@@ -507,10 +525,9 @@ int sm_count() {
 // Stats -> mu -> encode for one append, statistics in `sc` (words already zeroed).
 // The token splits of the stats pass fill one wave of resident CTAs (at most
 // kSplits, the size the scratch is laid out for).
-cudaError_t launch_append_kernels(const KVLayout& L, const void* k, const void* v, int32_t slot,
+cudaError_t launch_append_kernels(const KVLayout& L, const void* k, const void* v, int64_t T, int32_t slot,
                                   const Scratch& sc, unsigned* status, cudaStream_t s) {
   const int64_t C = (int64_t)L.heads * L.head_dim;
-  const int64_t T = L.chunk_tokens;
   static int resident[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -559,11 +576,11 @@ cudaError_t launch_append_kernels(const KVLayout& L, const void* k, const void* 
   ep.k_scales = L.base + L.off_k_scales + (int64_t)slot * L.slot_scales_bytes;
   ep.v_scales = L.base + L.off_v_scales + (int64_t)slot * L.slot_scales_bytes;
   ep.gscale = reinterpret_cast<float*>(L.base + L.off_gscale) + 2 * (int64_t)slot;
+  ep.slot_tokens = reinterpret_cast<int32_t*>(L.base + L.off_tokens) + slot;
+  ep.tokens = (int32_t)T;
   ep.words = sc.words;
   ep.status = status;
-  const int64_t want = (ep.nblocks + kEncThreads - 1) / kEncThreads;
-  const int64_t cap = (int64_t)sm_count() * 8;
-  kv_encode_kernel<<<(unsigned)(want < cap ? want : cap), kEncThreads, 0, s>>>(ep);
+  kv_encode_kernel<<<wave_grid<kv_encode_kernel>(kEncThreads, ep.nblocks), kEncThreads, 0, s>>>(ep);
   return cudaGetLastError();
 }
 
@@ -575,18 +592,18 @@ int64_t kv_scratch_bytes(int32_t heads, int32_t head_dim, int64_t chunk_tokens) 
   return align256((int64_t)kSplits * C * 8) + 3 * align256((int64_t)kSplits * C * 4) + 256;
 }
 
-cudaError_t launch_kv_append(const KVLayout& L, const void* k, const void* v, int32_t slot,
+cudaError_t launch_kv_append(const KVLayout& L, const void* k, const void* v, int64_t tokens, int32_t slot,
                              unsigned* status, cudaStream_t s) {
   const int64_t C = (int64_t)L.heads * L.head_dim;
   Scratch sc = scratch_at(L.base + L.off_scratch, C);
   cudaError_t e = cudaMemsetAsync(sc.words, 0, 3 * sizeof(unsigned), s);
   if (e != cudaSuccess) return e;
 
-  return launch_append_kernels(L, k, v, slot, sc, status, s);
+  return launch_append_kernels(L, k, v, tokens, slot, sc, status, s);
 }
 
-cudaError_t launch_kv_window(const KVLayout& L, const int32_t* slots, int32_t n_slots, void* k_out,
-                             void* v_out, cudaStream_t s) {
+cudaError_t launch_kv_window(const KVLayout& L, const int32_t* slots, const int32_t* tokens, int32_t n_slots,
+                             void* k_out, void* v_out, unsigned* status, cudaStream_t s) {
   WindowParams p;
   p.base = L.base;
   p.off_k_codes = L.off_k_codes;
@@ -595,19 +612,24 @@ cudaError_t launch_kv_window(const KVLayout& L, const int32_t* slots, int32_t n_
   p.off_v_scales = L.off_v_scales;
   p.off_mu = L.off_mu;
   p.off_gscale = L.off_gscale;
+  p.off_tokens = L.off_tokens;
   p.slot_codes_bytes = L.slot_codes_bytes;
   p.slot_scales_bytes = L.slot_scales_bytes;
   p.C = (int64_t)L.heads * L.head_dim;
-  p.blocks_per_chunk = L.chunk_tokens * p.C / 16;
-  p.bpc = FastDiv((uint32_t)p.blocks_per_chunk);
   p.cblocks = FastDiv((uint32_t)(p.C / 16));
-  p.nblocks = (int64_t)n_slots * p.blocks_per_chunk;
-  for (int i = 0; i < kMaxWindow; ++i) p.slots[i] = i < n_slots ? slots[i] : 0;
-  p.k_out = (uint8_t*)k_out;
-  p.v_out = (uint8_t*)v_out;
-  const int64_t want = (2 * p.nblocks + kEncThreads - 1) / kEncThreads;
-  const int64_t cap = (int64_t)sm_count() * 8;
-  kv_window_kernel<<<(unsigned)(want < cap ? want : cap), kEncThreads, 0, s>>>(p);
+  int64_t acc = 0;
+  p.n_slots = n_slots;
+  for (int i = 0; i < n_slots; ++i) {
+    p.slots[i] = slots[i];
+    p.tokens[i] = tokens[i];
+    acc += (int64_t)tokens[i] * p.C / 8;
+    p.hb_end[i] = acc;
+  }
+  p.k_out = static_cast<uint8_t*>(k_out);
+  p.v_out = static_cast<uint8_t*>(v_out);
+  p.status = status;
+  const int grid = wave_grid<kv_window_kernel>(kEncThreads, acc);
+  kv_window_kernel<<<grid, kEncThreads, 0, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -646,8 +668,8 @@ static cudaError_t kv_noalloc_scratch(uint8_t** out) {
   return cudaSuccess;
 }
 
-cudaError_t launch_kv_append_noalloc(const KVLayout& L, const void* k, const void* v, int32_t slot,
-                                     unsigned* status, cudaStream_t s) {
+cudaError_t launch_kv_append_noalloc(const KVLayout& L, const void* k, const void* v, int64_t tokens,
+                                     int32_t slot, unsigned* status, cudaStream_t s) {
   const int64_t C = (int64_t)L.heads * L.head_dim;
   if (C > kNoAllocMaxColumns) return cudaErrorInvalidValue;
   uint8_t* scratch = nullptr;
@@ -658,7 +680,7 @@ cudaError_t launch_kv_append_noalloc(const KVLayout& L, const void* k, const voi
   // statistics of every split in use are fully rewritten by kv_stats_kernel
   if ((e = cudaMemsetAsync(sc.words, 0, 3 * sizeof(unsigned), s)) != cudaSuccess) return e;
 
-  return launch_append_kernels(L, k, v, slot, sc, status, s);
+  return launch_append_kernels(L, k, v, tokens, slot, sc, status, s);
 }
 
 }  // namespace nvfp4

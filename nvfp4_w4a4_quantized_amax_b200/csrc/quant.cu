@@ -211,14 +211,6 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantParams p) {
   }
 }
 
-int grid_for(int64_t work) {
-  int dev = 0, sms = 148;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int64_t want = (work + kThreads - 1) / kThreads;
-  const int64_t cap = (int64_t)sms * 8;
-  return (int)(want < cap ? (want > 0 ? want : 1) : cap);
-}
 
 }  // namespace
 
@@ -240,10 +232,10 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
     const int64_t cpr = a.cols * esz / 16;
     const int64_t n = a.rows * cpr;
     if (a.x_bf16)
-      amax_kernel<true><<<grid_for(n), kThreads, 0, s>>>((const uint8_t*)a.x, a.ldx * esz, n,
+      amax_kernel<true><<<wave_grid<amax_kernel<true>>(kThreads, n), kThreads, 0, s>>>((const uint8_t*)a.x, a.ldx * esz, n,
                                                          FastDiv((uint32_t)cpr), amax_bits);
     else
-      amax_kernel<false><<<grid_for(n), kThreads, 0, s>>>((const uint8_t*)a.x, a.ldx * esz, n,
+      amax_kernel<false><<<wave_grid<amax_kernel<false>>(kThreads, n), kThreads, 0, s>>>((const uint8_t*)a.x, a.ldx * esz, n,
                                                           FastDiv((uint32_t)cpr), amax_bits);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -267,13 +259,13 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
   p.gscale_out = a.gscale_out;
   p.amax_accum = a.gscale_in ? amax_bits : nullptr;
   p.status = a.status;
-  const int grid = grid_for(p.nvblocks);
+  const int64_t n = p.nvblocks;
   if (a.x_bf16) {
-    if (a.sf_mma) encode_kernel<true, true><<<grid, kThreads, 0, s>>>(p);
-    else encode_kernel<true, false><<<grid, kThreads, 0, s>>>(p);
+    if (a.sf_mma) encode_kernel<true, true><<<wave_grid<encode_kernel<true, true>>(kThreads, n), kThreads, 0, s>>>(p);
+    else encode_kernel<true, false><<<wave_grid<encode_kernel<true, false>>(kThreads, n), kThreads, 0, s>>>(p);
   } else {
-    if (a.sf_mma) encode_kernel<false, true><<<grid, kThreads, 0, s>>>(p);
-    else encode_kernel<false, false><<<grid, kThreads, 0, s>>>(p);
+    if (a.sf_mma) encode_kernel<false, true><<<wave_grid<encode_kernel<false, true>>(kThreads, n), kThreads, 0, s>>>(p);
+    else encode_kernel<false, false><<<wave_grid<encode_kernel<false, false>>(kThreads, n), kThreads, 0, s>>>(p);
   }
   return cudaGetLastError();
 }
@@ -292,13 +284,13 @@ cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t s) {
   p.nb_per_row = FastDiv((uint32_t)nb);
   p.y = (uint8_t*)a.y;
   p.y_row_bytes = a.ldy * (a.y_bf16 ? 2 : 4);
-  const int grid = grid_for(2 * p.nblocks);
+  const int64_t n = 2 * p.nblocks;
   if (a.sf_mma) {
-    if (a.y_bf16) dequant_kernel<true, true><<<grid, kThreads, 0, s>>>(p);
-    else dequant_kernel<true, false><<<grid, kThreads, 0, s>>>(p);
+    if (a.y_bf16) dequant_kernel<true, true><<<wave_grid<dequant_kernel<true, true>>(kThreads, n), kThreads, 0, s>>>(p);
+    else dequant_kernel<true, false><<<wave_grid<dequant_kernel<true, false>>(kThreads, n), kThreads, 0, s>>>(p);
   } else {
-    if (a.y_bf16) dequant_kernel<false, true><<<grid, kThreads, 0, s>>>(p);
-    else dequant_kernel<false, false><<<grid, kThreads, 0, s>>>(p);
+    if (a.y_bf16) dequant_kernel<false, true><<<wave_grid<dequant_kernel<false, true>>(kThreads, n), kThreads, 0, s>>>(p);
+    else dequant_kernel<false, false><<<wave_grid<dequant_kernel<false, false>>(kThreads, n), kThreads, 0, s>>>(p);
   }
   return cudaGetLastError();
 }

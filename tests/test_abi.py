@@ -100,9 +100,10 @@ def test_host_argument_checks_return_before_any_device_work():
         nv.ERR_ALIGNMENT
     assert lib.nvfp4_kv_cache_init(ctypes.c_void_p(4096), 16, 2, 16, 64, 2, ctypes.byref(h)) == nv.ERR_SHAPE
     assert lib.nvfp4_kv_cache_init(ctypes.c_void_p(4096), 1 << 30, 2, 16, 64, 2, ctypes.byref(h)) == nv.OK
-    # append: wrong token count, slot out of range; window: empty list
-    assert lib.kv_quant_append(ctypes.byref(h), ctypes.c_void_p(4096), ctypes.c_void_p(4096), 63, 0,
-                               None) == nv.ERR_SHAPE
+    # append: token count outside 1..chunk_tokens, slot out of range; window: empty list
+    for bad_tokens in (0, 65, -1):
+        assert lib.kv_quant_append(ctypes.byref(h), ctypes.c_void_p(4096), ctypes.c_void_p(4096), bad_tokens,
+                                   0, None) == nv.ERR_SHAPE
     assert lib.kv_quant_append(ctypes.byref(h), ctypes.c_void_p(4096), ctypes.c_void_p(4096), 64, 2,
                                None) == nv.ERR_INVALID_ARG
     slots = (ctypes.c_int32 * 1)(5)
@@ -110,3 +111,15 @@ def test_host_argument_checks_return_before_any_device_work():
                                  ctypes.c_void_p(4096), None) == nv.ERR_INVALID_ARG
     assert lib.kv_dequant_window(ctypes.byref(h), slots, 0, ctypes.c_void_p(4096),
                                  ctypes.c_void_p(4096), None) == nv.ERR_INVALID_ARG
+    # token windows: missing counts, counts outside 1..chunk_tokens, bad slot, too many slots
+    ok_slots = (ctypes.c_int32 * 2)(0, 1)
+    W = lib.kv_dequant_window_tokens
+    out = ctypes.c_void_p(4096)
+    assert W(ctypes.byref(h), ok_slots, None, 2, out, out, None) == nv.ERR_INVALID_ARG
+    for bad in ((0, 64), (64, 65), (-3, 1)):
+        toks = (ctypes.c_int32 * 2)(*bad)
+        assert W(ctypes.byref(h), ok_slots, toks, 2, out, out, None) == nv.ERR_SHAPE
+    toks = (ctypes.c_int32 * 2)(64, 17)
+    assert W(ctypes.byref(h), (ctypes.c_int32 * 2)(0, 2), toks, 2, out, out, None) == nv.ERR_INVALID_ARG
+    many = (ctypes.c_int32 * 65)(*([0] * 65))
+    assert W(ctypes.byref(h), many, many, 65, out, out, None) == nv.ERR_INVALID_ARG

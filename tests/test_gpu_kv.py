@@ -108,3 +108,74 @@ def test_full_size_cache_24x128_8192_tokens(cuda_dev):
     """24 heads x 128, chunks of 8192 tokens: 5 appends (every slot checked) and a
     4-chunk window of 32768 tokens, all values compared."""
     run_cache(heads=24, head_dim=128, T=8192, chunks=5, window=4, seed=3)
+
+
+def check_slot_prefix(cache, slot, ref):
+    """A slot holding ref.T tokens (possibly fewer than chunk_tokens): its first tokens."""
+    kc, ks, vc, vs, mu, g = cache.slot_views(slot)
+    C = ref.H * ref.Dh
+    nc, ns = ref.T * C // 2, ref.T * C // 16
+    assert cache.slot_tokens(slot) == ref.T
+    assert np.array_equal(mu.cpu().numpy().view(np.uint32), ref.mu.view(np.uint32)), "mu"
+    gk, gv = g.cpu().numpy().tolist()
+    assert gk == ref.g_k and gv == ref.g_v
+    assert np.array_equal(kc[:nc].cpu().numpy(), ref.k_codes.ravel()), "K codes"
+    assert np.array_equal(ks[:ns].cpu().numpy(), ref.k_scales.ravel()), "K scales"
+    assert np.array_equal(vc[:nc].cpu().numpy(), ref.v_codes.ravel()), "V codes"
+    assert np.array_equal(vs[:ns].cpu().numpy(), ref.v_scales.ravel()), "V scales"
+
+
+def test_partial_chunks_and_sink_aware_window(cuda_dev):
+    """Slots holding 17, 1, 1000, 333 and all 2048 tokens; a sink-aware window lists a
+    sink slot, a shot-sink slot, the sliding slots (one partial) and a repeat."""
+    heads, hd, T = 4, 64, 2048
+    off = synth.kv_offsets(9, heads, hd)
+    cache = nv.KVCache(heads, hd, T, 6)
+    fills = {0: 17, 1: T, 2: 1, 3: 1000, 4: T, 5: 333}
+    refs = {}
+    for slot, n in fills.items():
+        k, v = synth.kv_chunk(9, slot, T, heads, hd, off)
+        k, v = np.ascontiguousarray(k[:n]), np.ascontiguousarray(v[:n])
+        nv.kv_quant_append(cache, dev_bf16(k), dev_bf16(v), slot)
+        refs[slot] = oracle.kv_append(k, v)
+        torch.cuda.synchronize()
+        check_slot_prefix(cache, slot, refs[slot])
+    slots = [0, 2, 3, 4, 5, 1, 3]
+    toks = [fills[s] for s in slots]
+    ko = torch.full((sum(toks), heads, hd), float("nan"), dtype=torch.bfloat16, device="cuda")
+    vo = torch.full_like(ko, float("nan"))
+    nv.kv_dequant_window_tokens(cache, slots, toks, ko, vo)
+    kh, vh = host_bits(ko), host_bits(vo)
+    row = 0
+    for s, n in zip(slots, toks):
+        rk, rv = oracle.kv_dequant_chunk(refs[s])
+        assert np.array_equal(kh[row:row + n], rk), f"K^ slot {s}"
+        assert np.array_equal(vh[row:row + n], rv), f"V^ slot {s}"
+        row += n
+    assert device_status() == nv.OK
+
+
+def test_window_token_count_mismatch_sets_status_and_skips_the_slot(cuda_dev):
+    heads, hd, T = 2, 32, 256
+    off = synth.kv_offsets(10, heads, hd)
+    cache = nv.KVCache(heads, hd, T, 2)
+    k, v = synth.kv_chunk(10, 0, T, heads, hd, off)
+    nv.kv_quant_append(cache, dev_bf16(k[:100].copy()), dev_bf16(v[:100].copy()), 0)
+    nv.kv_quant_append(cache, dev_bf16(k), dev_bf16(v), 1)
+    ref1 = oracle.kv_append(k, v)
+    torch.cuda.synchronize()
+    assert device_status(clear=True) == nv.OK
+    sentinel = 0x7F7F
+    ko = torch.full((T + 99, heads, hd), 0, dtype=torch.int16, device="cuda").fill_(sentinel).view(torch.bfloat16)
+    vo = torch.full((T + 99, heads, hd), 0, dtype=torch.int16, device="cuda").fill_(sentinel).view(torch.bfloat16)
+    nv.kv_dequant_window_tokens(cache, [1, 0], [T, 99], ko, vo)  # slot 0 holds 100, not 99
+    assert device_status(clear=True) == nv.ERR_SHAPE
+    kh, vh = host_bits(ko), host_bits(vo)
+    rk, rv = oracle.kv_dequant_chunk(ref1)
+    assert np.array_equal(kh[:T], rk) and np.array_equal(vh[:T], rv)
+    assert np.all(kh[T:] == sentinel) and np.all(vh[T:] == sentinel)
+    # the full-chunk window reports a partial slot the same way
+    k2 = torch.empty((T, heads, hd), dtype=torch.bfloat16, device="cuda")
+    nv.kv_dequant_window(cache, [0], k2, torch.empty_like(k2))
+    assert device_status(clear=True) == nv.ERR_SHAPE
+    assert device_status() == nv.OK
