@@ -76,6 +76,8 @@ def _load():
             lib.oracle_gelu_tanh.restype = dbl
             lib.oracle_gelu_tanh.argtypes = [dbl]
             lib.oracle_gelu_tanh_array.argtypes = [vp, i64, vp]
+            lib.oracle_lora_merge.restype = None
+            lib.oracle_lora_merge.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, vp, i64, f32, vp, i64]
             _lib = lib
     return _lib
 
@@ -260,4 +262,23 @@ def gelu_tanh(c: np.ndarray) -> np.ndarray:
     c = np.ascontiguousarray(c, dtype=np.float32)
     out = np.zeros(c.shape, dtype=np.float64)
     _load().oracle_gelu_tanh_array(_p(c), c.size, _p(out))
+    return out
+
+
+def lora_merge(w: np.ndarray, b: np.ndarray, a: np.ndarray, scale: float) -> np.ndarray:
+    """W' = W + scale * (B A) in binary32 with the oracle's fixed order (see
+    oracle_lora_merge).  w: uint16 (bf16 bits) or float32 [rows, cols];
+    b: float32 [rows, rank]; a: float32 [rank, cols].  Returns float32 [rows, cols]."""
+    w = np.ascontiguousarray(w)
+    wt = 0 if w.dtype == np.uint16 else 1
+    if wt == 1:
+        w = w.astype(np.float32, copy=False)
+    b = np.ascontiguousarray(b, dtype=np.float32)
+    a = np.ascontiguousarray(a, dtype=np.float32)
+    rows, cols = w.shape
+    rank = b.shape[1]
+    assert b.shape == (rows, rank) and a.shape == (rank, cols)
+    out = np.zeros((rows, cols), np.float32)
+    _load().oracle_lora_merge(_p(w), wt, rows, cols, cols, _p(b), _p(a), rank, float(np.float32(scale)), _p(out),
+                              cols)
     return out

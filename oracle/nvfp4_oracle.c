@@ -371,3 +371,32 @@ double oracle_gelu_tanh(double c) {
 void oracle_gelu_tanh_array(const float* c, int64_t n, double* out) {
   for (int64_t i = 0; i < n; ++i) out[i] = oracle_gelu_tanh((double)c[i]);
 }
+
+/* ---------------------------------------------------------------- LoRA merge */
+
+/* A LoRA update merged into a weight before the weight is quantized.
+ * [ZD] github.zuobiaodaohang.com, "长视频生成的两堵物理墙", section "NVFP4：数据体积砍到
+ * 1/4", further optimizations: "LoRA before quantization" (the LoRA is loaded into
+ * the weight first, then the weight is quantized, for accuracy).
+ * Reading (the page gives no formula): the usual LoRA update
+ *   W' = W + scale * (B A),  B [rows, rank], A [rank, cols],
+ * in binary32 with one fixed order of operations:
+ *   acc = 0;  for j = 0 .. rank-1:  acc = RN(acc + RN(B[r][j] * A[j][c]));
+ *   W'[r][c] = RN(W[r][c] + RN(scale * acc)).
+ * W is bf16 bits (wt 0) or float (wt 1), row pitch ldw elements; B has row pitch
+ * rank, A row pitch cols; out is float [rows, cols] with row pitch ldo.  Non-finite
+ * values propagate (quantizing the result reports them). */
+void oracle_lora_merge(const void* w, int wt, int64_t rows, int64_t cols, int64_t ldw, const float* b,
+                       const float* a, int64_t rank, float scale, float* out, int64_t ldo) {
+  for (int64_t r = 0; r < rows; ++r) {
+    for (int64_t c = 0; c < cols; ++c) {
+      float acc = 0.0f;
+      for (int64_t j = 0; j < rank; ++j) {
+        const float p = b[r * rank + j] * a[j * cols + c];
+        acc = acc + p;
+      }
+      const float u = scale * acc;
+      out[r * ldo + c] = load_elem(w, wt, r * ldw + c) + u;
+    }
+  }
+}
