@@ -543,6 +543,15 @@ def run_single_kernel(args):
         y = torch.empty((R, C), dtype=torch.bfloat16, device=dev)
         fn = (lambda: nv.nvfp4_quantize(x, q, amax_out=amax[0:1])) if args.kernel == "quantize" else \
             (lambda: nv.nvfp4_dequantize(q, y))
+    elif args.kernel == "lora_merge":
+        # FFN-up weight 14336 x 3072 (bf16) + rank-64 LoRA -> FP32 W' (then quantized offline)
+        rows, cols, rank = 14336, 3072, 64
+        rng = np.random.default_rng(7)
+        w = to_dev(synth.weights(2, 2, rows, cols))
+        lb = torch.from_numpy((rng.standard_normal((rows, rank)) * 0.02).astype(np.float32)).to(dev)
+        la = torch.from_numpy((rng.standard_normal((rank, cols)) * 0.02).astype(np.float32)).to(dev)
+        out = torch.empty((rows, cols), dtype=torch.float32, device=dev)
+        fn = lambda: nv.nvfp4_lora_merge(w, lb, la, 2.0 / rank, out)  # noqa: E731
     elif args.kernel == "kv_window_sink":
         # sink-aware window: a 1024-token sink slot, a 4096-token shot-sink slot, three
         # full sliding slots and the newest, partial slot (3000 tokens): 32696 tokens
@@ -593,7 +602,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel", default=None,
-                    help="profiling mode: gemm | gemm_fused | quantize | dequantize | kv_append | kv_window | kv_window_sink")
+                    help="profiling mode: gemm | gemm_fused | quantize | dequantize | kv_append | kv_window | kv_window_sink | lora_merge")
     ap.add_argument("--shape", default="8192,14336,3072", help="M,N,K for gemm; rows,cols for (de)quantize")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--kernel-warmup", type=int, default=1,

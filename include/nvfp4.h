@@ -269,6 +269,26 @@ nvfp4_status kv_dequant_window_tokens(const nvfp4_kv_cache* cache, const int32_t
                                       const int32_t* tokens_host, int32_t n_slots, void* k_out,
                                       void* v_out, nvfp4_stream_t stream);
 
+/* ------------------------------------------------------------- LoRA merge ----
+ * github.zuobiaodaohang.com, "长视频生成的两堵物理墙", section "NVFP4：数据体积砍到 1/4":
+ * "LoRA before quantization" — the LoRA is loaded into the weight first, then the
+ * weight is quantized.  Reading fixed here (the page gives no formula): the usual
+ * LoRA update in binary32 with one fixed order,
+ *   acc = 0;  for j = 0 .. rank-1:  acc = RN(acc + RN(B[r][j] * A[j][c]));
+ *   out[r][c] = RN(W[r][c] + RN(scale * acc)),
+ * and the caller quantizes `out` with nvfp4_quantize (NVFP4_FP32 input).
+ * nvfp4_lora_merge:
+ *   w     : device [rows][ldw] of type wt (bf16 or fp32), ldw >= cols.
+ *   lora_b: device fp32 [rows][rank] (row pitch rank);  lora_a: device fp32
+ *           [rank][cols] (row pitch cols);  1 <= rank <= 4096.
+ *   out   : device fp32 [rows][ldo], ldo >= cols; may not overlap w, lora_a or lora_b.
+ * Errors: NULL pointers or rank outside 1..4096 -> INVALID_ARG; negative sizes or
+ * pitches below cols -> SHAPE.  Non-finite values propagate into out (quantizing
+ * it reports them).  rows == 0 or cols == 0 does nothing. */
+nvfp4_status nvfp4_lora_merge(const void* w, nvfp4_dtype wt, int64_t rows, int64_t cols, int64_t ldw,
+                              const float* lora_b, const float* lora_a, int32_t rank, float scale,
+                              float* out, int64_t ldo, nvfp4_stream_t stream);
+
 /* ----------------------------------------------------------------- status ----
  * Reads the sticky device status word of CUDA device `device` (synchronizes that
  * device first).  *status_out is NVFP4_OK or the first data error recorded since

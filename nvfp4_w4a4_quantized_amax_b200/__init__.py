@@ -64,6 +64,7 @@ class nvfp4_kv_cache(ctypes.Structure):
 EXPORTS = ["nvfp4_version", "nvfp4_status_string", "nvfp4_scales_bytes", "nvfp4_quantize",
            "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_cache_bytes", "nvfp4_kv_cache_init",
            "kv_quant_append", "kv_quant_append_noalloc", "kv_dequant_window", "kv_dequant_window_tokens",
+           "nvfp4_lora_merge",
            "nvfp4_get_device_status"]
 
 
@@ -103,6 +104,8 @@ def library():
             lib.kv_dequant_window_tokens.restype = i32
             lib.kv_dequant_window_tokens.argtypes = [KV, ctypes.POINTER(ctypes.c_int32),
                                                      ctypes.POINTER(ctypes.c_int32), i32, vp, vp, vp]
+            lib.nvfp4_lora_merge.restype = i32
+            lib.nvfp4_lora_merge.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32, ctypes.c_float, vp, i64, vp]
             lib.nvfp4_get_device_status.restype = i32
             lib.nvfp4_get_device_status.argtypes = [i32, ctypes.POINTER(ctypes.c_int32), i32]
             _lib = lib
@@ -280,6 +283,17 @@ def kv_dequant_window_tokens(cache: KVCache, slots: Sequence[int], tokens: Seque
     tarr = (ctypes.c_int32 * len(tokens))(*tokens)
     _check(library().kv_dequant_window_tokens(ctypes.byref(cache.handle), sarr, tarr, len(slots), _ptr(k_out),
                                               _ptr(v_out), _stream(stream)), "kv_dequant_window_tokens")
+
+
+def nvfp4_lora_merge(w, lora_b, lora_a, scale: float, out, stream=None):
+    """out = W + scale * (B A) in binary32 with the library's fixed order (LoRA merged
+    before quantization).  w: bf16 or fp32 [rows, cols]; lora_b fp32 [rows, rank];
+    lora_a fp32 [rank, cols]; out fp32 [rows, cols]."""
+    rows, cols = w.shape
+    rank = lora_b.shape[1]
+    _check(library().nvfp4_lora_merge(_ptr(w), _dtype_code(w), rows, cols, w.stride(0), _ptr(lora_b),
+                                      _ptr(lora_a), rank, float(scale), _ptr(out), out.stride(0),
+                                      _stream(stream)), "nvfp4_lora_merge")
 
 
 def get_device_status(device: int = 0, clear: bool = False) -> int:

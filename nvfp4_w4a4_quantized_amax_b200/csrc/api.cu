@@ -359,6 +359,33 @@ nvfp4_status kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t* slots
   return kv_dequant_window_tokens(cache, slots_host, tokens, n_slots, k_out, v_out, stream);
 }
 
+nvfp4_status nvfp4_lora_merge(const void* w, nvfp4_dtype wt, int64_t rows, int64_t cols, int64_t ldw,
+                              const float* lora_b, const float* lora_a, int32_t rank, float scale,
+                              float* out, int64_t ldo, nvfp4_stream_t stream) {
+  if (!valid_dtype(wt) || rank < 1 || rank > 4096) return NVFP4_ERR_INVALID_ARG;
+  if (rows < 0 || cols < 0) return NVFP4_ERR_SHAPE;
+  if (rows == 0 || cols == 0) return NVFP4_OK;
+  if (!w || !lora_b || !lora_a || !out) return NVFP4_ERR_INVALID_ARG;
+  if (ldw < cols || ldo < cols) return NVFP4_ERR_SHAPE;
+  if (rows > (int64_t)1 << 31 || cols > (int64_t)1 << 31) return NVFP4_ERR_SHAPE;
+  unsigned* status = nullptr;
+  nvfp4_status st = current_device(&status);
+  if (st != NVFP4_OK) return st;
+  nvfp4::LoraArgs a;
+  a.w = w;
+  a.w_bf16 = wt == NVFP4_BF16;
+  a.rows = rows;
+  a.cols = cols;
+  a.ldw = ldw;
+  a.b = lora_b;
+  a.a = lora_a;
+  a.rank = rank;
+  a.scale = scale;
+  a.out = out;
+  a.ldo = ldo;
+  return cuda_status(nvfp4::launch_lora_merge(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_get_device_status(int32_t device, int32_t* status_out, int32_t clear) {
   if (!status_out) return NVFP4_ERR_INVALID_ARG;
   int prev = 0;

@@ -86,6 +86,19 @@ constexpr int kMaxWindowSlots = 64;
 cudaError_t launch_kv_window(const KVLayout& c, const int32_t* slots, const int32_t* tokens, int32_t n_slots,
                              void* k_out, void* v_out, unsigned* status, cudaStream_t s);
 
+struct LoraArgs {
+  const void* w;   // bf16 or fp32 [rows][ldw]
+  bool w_bf16;
+  int64_t rows, cols, ldw;
+  const float* b;  // [rows][rank]
+  const float* a;  // [rank][cols]
+  int64_t rank;
+  float scale;
+  float* out;      // [rows][ldo]
+  int64_t ldo;
+};
+cudaError_t launch_lora_merge(const LoraArgs& a, cudaStream_t s);
+
 struct GemmOperand {
   const uint8_t* codes;
   int64_t ld_codes;

@@ -123,3 +123,12 @@ def test_host_argument_checks_return_before_any_device_work():
     assert W(ctypes.byref(h), (ctypes.c_int32 * 2)(0, 2), toks, 2, out, out, None) == nv.ERR_INVALID_ARG
     many = (ctypes.c_int32 * 65)(*([0] * 65))
     assert W(ctypes.byref(h), many, many, 65, out, out, None) == nv.ERR_INVALID_ARG
+    # LoRA merge: rank outside 1..4096, NULL factors, pitch below cols; empty is a no-op
+    L = lib.nvfp4_lora_merge
+    p = ctypes.c_void_p(4096)
+    assert L(p, nv.BF16, 4, 32, 32, p, p, 0, 1.0, p, 32, None) == nv.ERR_INVALID_ARG
+    assert L(p, nv.BF16, 4, 32, 32, p, p, 4097, 1.0, p, 32, None) == nv.ERR_INVALID_ARG
+    assert L(p, nv.BF16, 4, 32, 32, None, p, 8, 1.0, p, 32, None) == nv.ERR_INVALID_ARG
+    assert L(p, nv.BF16, 4, 32, 16, p, p, 8, 1.0, p, 32, None) == nv.ERR_SHAPE
+    assert L(p, 7, 4, 32, 32, p, p, 8, 1.0, p, 32, None) == nv.ERR_INVALID_ARG
+    assert L(None, nv.BF16, 0, 32, 32, None, None, 8, 1.0, None, 32, None) == nv.OK
