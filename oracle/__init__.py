@@ -76,6 +76,8 @@ def _load():
             lib.oracle_gelu_tanh.restype = dbl
             lib.oracle_gelu_tanh.argtypes = [dbl]
             lib.oracle_gelu_tanh_array.argtypes = [vp, i64, vp]
+            lib.oracle_amax_history_push.restype = ctypes.c_int
+            lib.oracle_amax_history_push.argtypes = [vp, i64, f32, vp]
             lib.oracle_lora_merge.restype = None
             lib.oracle_lora_merge.argtypes = [vp, ctypes.c_int, i64, i64, i64, vp, vp, i64, f32, vp, i64]
             _lib = lib
@@ -282,3 +284,14 @@ def lora_merge(w: np.ndarray, b: np.ndarray, a: np.ndarray, scale: float) -> np.
     _load().oracle_lora_merge(_p(w), wt, rows, cols, cols, _p(b), _p(a), rank, float(np.float32(scale)), _p(out),
                               cols)
     return out
+
+
+def amax_history_push(history: np.ndarray, amax_new: float):
+    """(updated history, g) after pushing amax_new (see oracle_amax_history_push);
+    raises on a non-finite amax_new."""
+    h = np.ascontiguousarray(history, dtype=np.float32).copy()
+    g = np.zeros(1, np.float32)
+    st = _load().oracle_amax_history_push(_p(h), h.size, float(np.float32(amax_new)), _p(g))
+    if st != 0:
+        raise ValueError("non-finite amax")
+    return h, float(g[0])

@@ -400,3 +400,23 @@ void oracle_lora_merge(const void* w, int wt, int64_t rows, int64_t cols, int64_
     }
   }
 }
+
+/* ------------------------------------------------------- amax history (C8) */
+
+/* Tensor scale of a requantizing GEMM epilogue from the max|h| of earlier calls.
+ * The epilogue quantizes before its own max|h| is known, so it takes a supplied
+ * scale; reading fixed here: keep the last len values of max|h| (newest first)
+ * and supply g = RN(max(history) / 2688), the tensor-scale formula of quantize.
+ * Push: history[i] = history[i-1] for i = len-1 .. 1, history[0] = amax_new, then
+ * *g_out from the updated history.  A non-finite amax_new changes nothing and
+ * returns ORACLE_ERR_NONFINITE. */
+int oracle_amax_history_push(float* history, int64_t len, float amax_new, float* g_out) {
+  if (!(fabsf(amax_new) <= 3.402823466e38f)) return ORACLE_ERR_NONFINITE;
+  for (int64_t i = len - 1; i >= 1; --i) history[i] = history[i - 1];
+  history[0] = amax_new;
+  float m = 0.0f;
+  for (int64_t i = 0; i < len; ++i)
+    if (history[i] > m) m = history[i];
+  *g_out = m / 2688.0f;
+  return ORACLE_OK;
+}
