@@ -204,10 +204,14 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     vo = torch.empty_like(ko)
     amax = torch.zeros(8, dtype=torch.float32, device=dev)
 
-    # calibration of the fused FFN's supplied tensor scale (one earlier chunk)
+    # supplied tensor scale of the fused FFN's requantization: an amax history of
+    # the FFN-up output (16 chunks), started by one calibration chunk and updated
+    # by every step with that step's max|h|
     nv.nvfp4_quantize(x5, qx5, amax_out=amax[4:5])
     nv.nvfp4_gemm(qx5, q1, None, act=nv.ACT_GELU_TANH, q_amax_out=amax[5:6])
-    g_h = (amax[5:6] / 2688.0).contiguous()
+    hist = torch.zeros(16, dtype=torch.float32, device=dev)
+    g_h = torch.zeros(1, dtype=torch.float32, device=dev)
+    nv.nvfp4_amax_history_push(hist, amax[5:6], g_h)
     for s in range(SLOTS):  # fill the cache
         k, v = kvd[s % 2]
         nv.kv_quant_append(cache, k, v, s)
@@ -249,6 +253,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         timed("gemm_ffn_up_gelu_requant", lambda: nv.nvfp4_gemm(qx5, q1, None, act=nv.ACT_GELU_TANH,
                                                                 q_out=qh, q_gscale_in=g_h,
                                                                 q_amax_out=amax[6:7]), 1, events)
+        timed("amax_history_push", lambda: nv.nvfp4_amax_history_push(hist, amax[6:7], g_h), 1, events)
         timed("gemm_ffn_down_bf16", lambda: nv.nvfp4_gemm(qh, q2, y5), 1, events)
 
     dist = None

@@ -269,6 +269,22 @@ nvfp4_status kv_dequant_window_tokens(const nvfp4_kv_cache* cache, const int32_t
                                       const int32_t* tokens_host, int32_t n_slots, void* k_out,
                                       void* v_out, nvfp4_stream_t stream);
 
+/* ----------------------------------------------------------- amax history ----
+ * A requantizing GEMM epilogue (nvfp4_epilogue.q_out) quantizes before its own
+ * max|h| is known, so it takes a supplied tensor scale (q_gscale_in) and reports
+ * max|h| (q_amax_out).  Reading fixed here for the steady state of chunk-by-chunk
+ * generation ([TW] §三: chunks are generated one after another with the same
+ * layers): keep the last `len` values of max|h| of a layer, newest first, and
+ * supply g = RN(max(history) / 2688), the tensor-scale formula of quantize.
+ * nvfp4_amax_history_push:
+ *   history    : device fp32 [len], 1 <= len <= 1024 (zeros before the first push).
+ *   amax_new   : device fp32, e.g. the previous call's q_amax_out.
+ *   gscale_out : device fp32, the scale for the next call's q_gscale_in.
+ * Shifts history by one, stores *amax_new in history[0], writes *gscale_out.  A
+ * non-finite *amax_new sets device status NONFINITE and changes nothing. */
+nvfp4_status nvfp4_amax_history_push(float* history, int32_t len, const float* amax_new, float* gscale_out,
+                                     nvfp4_stream_t stream);
+
 /* ------------------------------------------------------------- LoRA merge ----
  * github.zuobiaodaohang.com, "长视频生成的两堵物理墙", section "NVFP4：数据体积砍到 1/4":
  * "LoRA before quantization" — the LoRA is loaded into the weight first, then the

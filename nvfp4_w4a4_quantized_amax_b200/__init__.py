@@ -64,7 +64,7 @@ class nvfp4_kv_cache(ctypes.Structure):
 EXPORTS = ["nvfp4_version", "nvfp4_status_string", "nvfp4_scales_bytes", "nvfp4_quantize",
            "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_cache_bytes", "nvfp4_kv_cache_init",
            "kv_quant_append", "kv_quant_append_noalloc", "kv_dequant_window", "kv_dequant_window_tokens",
-           "nvfp4_lora_merge",
+           "nvfp4_lora_merge", "nvfp4_amax_history_push",
            "nvfp4_get_device_status"]
 
 
@@ -106,6 +106,8 @@ def library():
                                                      ctypes.POINTER(ctypes.c_int32), i32, vp, vp, vp]
             lib.nvfp4_lora_merge.restype = i32
             lib.nvfp4_lora_merge.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32, ctypes.c_float, vp, i64, vp]
+            lib.nvfp4_amax_history_push.restype = i32
+            lib.nvfp4_amax_history_push.argtypes = [vp, i32, vp, vp, vp]
             lib.nvfp4_get_device_status.restype = i32
             lib.nvfp4_get_device_status.argtypes = [i32, ctypes.POINTER(ctypes.c_int32), i32]
             _lib = lib
@@ -294,6 +296,13 @@ def nvfp4_lora_merge(w, lora_b, lora_a, scale: float, out, stream=None):
     _check(library().nvfp4_lora_merge(_ptr(w), _dtype_code(w), rows, cols, w.stride(0), _ptr(lora_b),
                                       _ptr(lora_a), rank, float(scale), _ptr(out), out.stride(0),
                                       _stream(stream)), "nvfp4_lora_merge")
+
+
+def nvfp4_amax_history_push(history, amax_new, gscale_out, stream=None):
+    """Shift amax_new (device fp32 [1]) into history (device fp32 [len]) and write the
+    next supplied tensor scale RN(max(history) / 2688) to gscale_out."""
+    _check(library().nvfp4_amax_history_push(_ptr(history), history.numel(), _ptr(amax_new), _ptr(gscale_out),
+                                             _stream(stream)), "nvfp4_amax_history_push")
 
 
 def get_device_status(device: int = 0, clear: bool = False) -> int:

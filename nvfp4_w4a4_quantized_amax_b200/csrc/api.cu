@@ -386,6 +386,17 @@ nvfp4_status nvfp4_lora_merge(const void* w, nvfp4_dtype wt, int64_t rows, int64
   return cuda_status(nvfp4::launch_lora_merge(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_amax_history_push(float* history, int32_t len, const float* amax_new, float* gscale_out,
+                                     nvfp4_stream_t stream) {
+  if (!history || !amax_new || !gscale_out) return NVFP4_ERR_INVALID_ARG;
+  if (len < 1 || len > nvfp4::kMaxHistory) return NVFP4_ERR_SHAPE;
+  unsigned* status = nullptr;
+  nvfp4_status st = current_device(&status);
+  if (st != NVFP4_OK) return st;
+  return cuda_status(nvfp4::launch_amax_history(history, len, amax_new, gscale_out, status,
+                                                reinterpret_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_get_device_status(int32_t device, int32_t* status_out, int32_t clear) {
   if (!status_out) return NVFP4_ERR_INVALID_ARG;
   int prev = 0;

@@ -212,6 +212,36 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantParams p) {
 }
 
 
+// Amax history of a requantizing epilogue (newest first): shift in *amax_new and
+// write g = RN(max(history) / 2688).  One CTA; a non-finite value changes nothing.
+constexpr int kHistThreads = 256;
+__global__ void __launch_bounds__(kHistThreads) amax_history_kernel(float* history, int len, const float* amax_new,
+                                                                   float* g_out, unsigned* status) {
+  __shared__ float old[kMaxHistory];
+  __shared__ unsigned red[kHistThreads / 32];
+  const float a = *amax_new;
+  if (!(fabsf(a) <= 3.402823466e38f)) {
+    if (threadIdx.x == 0) set_status(status, kStatusNonfinite);
+    return;
+  }
+  for (int i = threadIdx.x; i < len; i += kHistThreads) old[i] = history[i];
+  __syncthreads();
+  unsigned m = 0;  // max of non-negative floats as ordered bits
+  for (int i = threadIdx.x; i < len; i += kHistThreads) {
+    const float v = i == 0 ? a : old[i - 1];
+    history[i] = v;
+    m = max(m, __float_as_uint(fmaxf(v, 0.0f)));
+  }
+  m = warp_max_u32(m);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned mm = 0;
+    for (int w = 0; w < kHistThreads / 32; ++w) mm = max(mm, red[w]);
+    *g_out = __uint_as_float(mm) / 2688.0f;
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
@@ -295,4 +325,12 @@ cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+}  // namespace nvfp4
+
+namespace nvfp4 {
+cudaError_t launch_amax_history(float* history, int len, const float* amax_new, float* g_out, unsigned* status,
+                                cudaStream_t s) {
+  amax_history_kernel<<<1, kHistThreads, 0, s>>>(history, len, amax_new, g_out, status);
+  return cudaGetLastError();
+}
 }  // namespace nvfp4

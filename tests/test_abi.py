@@ -132,3 +132,8 @@ def test_host_argument_checks_return_before_any_device_work():
     assert L(p, nv.BF16, 4, 32, 16, p, p, 8, 1.0, p, 32, None) == nv.ERR_SHAPE
     assert L(p, 7, 4, 32, 32, p, p, 8, 1.0, p, 32, None) == nv.ERR_INVALID_ARG
     assert L(None, nv.BF16, 0, 32, 32, None, None, 8, 1.0, None, 32, None) == nv.OK
+    # amax history: NULL pointers, length outside 1..1024
+    Hp = lib.nvfp4_amax_history_push
+    assert Hp(None, 4, p, p, None) == nv.ERR_INVALID_ARG
+    assert Hp(p, 0, p, p, None) == nv.ERR_SHAPE
+    assert Hp(p, 1025, p, p, None) == nv.ERR_SHAPE
