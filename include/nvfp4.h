@@ -258,7 +258,9 @@ nvfp4_status kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t* slots
 /* kv_dequant_window_tokens — the same window over slots holding any number of
  * tokens, e.g. a sink-aware window: a sink slot, some shot-sink slots and the
  * sliding slots, possibly partial.  [TW] §四: one parallel kernel dequantizes the
- * window's chunks together.
+ * window's chunks together; [TW] §六: global and shot-level anchor frames stay in
+ * the attention range on top of the sliding window (a shot anchor is just a start
+ * and a length, nothing is copied).
  *   tokens_host : HOST array, tokens_host[i] = tokens held by slots_host[i]
  *                 (1 .. chunk_tokens).
  * Output: bf16 [sum(tokens_host)][heads][head_dim], the slots' tokens one after
