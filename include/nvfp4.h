@@ -319,6 +319,10 @@ const char* nvfp4_status_string(int32_t status);
 /* Library version, (major << 16) | minor. */
 int32_t nvfp4_version(void);
 
+/* Text of the CUDA error behind the last NVFP4_ERR_CUDA returned on the calling
+ * thread ("no error" if none); a static string owned by the CUDA runtime. */
+const char* nvfp4_last_cuda_error_string(void);
+
 #ifdef __cplusplus
 }
 #endif

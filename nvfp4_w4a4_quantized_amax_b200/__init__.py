@@ -33,7 +33,10 @@ _lib = None
 class Nvfp4Error(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {status_string(status)} (status {status})")
+        detail = ""
+        if status == ERR_CUDA:
+            detail = ": " + library().nvfp4_last_cuda_error_string().decode()
+        super().__init__(f"{where}: {status_string(status)} (status {status}){detail}")
 
 
 class nvfp4_tensor(ctypes.Structure):
@@ -64,7 +67,7 @@ class nvfp4_kv_cache(ctypes.Structure):
 EXPORTS = ["nvfp4_version", "nvfp4_status_string", "nvfp4_scales_bytes", "nvfp4_quantize",
            "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_cache_bytes", "nvfp4_kv_cache_init",
            "kv_quant_append", "kv_quant_append_noalloc", "kv_dequant_window", "kv_dequant_window_tokens",
-           "nvfp4_lora_merge", "nvfp4_amax_history_push",
+           "nvfp4_lora_merge", "nvfp4_amax_history_push", "nvfp4_last_cuda_error_string",
            "nvfp4_get_device_status"]
 
 
@@ -83,6 +86,8 @@ def library():
             lib.nvfp4_version.restype = i32
             lib.nvfp4_status_string.restype = ctypes.c_char_p
             lib.nvfp4_status_string.argtypes = [i32]
+            lib.nvfp4_last_cuda_error_string.restype = ctypes.c_char_p
+            lib.nvfp4_last_cuda_error_string.argtypes = []
             lib.nvfp4_scales_bytes.restype = i32
             lib.nvfp4_scales_bytes.argtypes = [i64, i64, i32, ctypes.POINTER(ctypes.c_size_t)]
             lib.nvfp4_quantize.restype = i32

@@ -50,7 +50,14 @@ nvfp4_status current_device(unsigned** status) {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-nvfp4_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVFP4_OK : NVFP4_ERR_CUDA; }
+// The CUDA error behind the last NVFP4_ERR_CUDA returned on this thread.
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+nvfp4_status cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return NVFP4_OK;
+  g_last_cuda_error = e;
+  return NVFP4_ERR_CUDA;
+}
 
 constexpr int64_t kMaxBlocks = (int64_t)1 << 31;
 
@@ -81,6 +88,10 @@ bool valid_dtype(int32_t t) { return t == NVFP4_BF16 || t == NVFP4_FP32; }
 extern "C" {
 
 int32_t nvfp4_version(void) { return (1 << 16) | 0; }
+
+const char* nvfp4_last_cuda_error_string(void) {
+  return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
+}
 
 const char* nvfp4_status_string(int32_t s) {
   switch (s) {
