@@ -313,6 +313,17 @@ nvfp4_status nvfp4_lora_merge(const void* w, nvfp4_dtype wt, int64_t rows, int64
  * the last clear; clear != 0 resets it to NVFP4_OK. */
 nvfp4_status nvfp4_get_device_status(int32_t device, int32_t* status_out, int32_t clear);
 
+/* Test hook for the bounded waits of the GEMM kernels (process-wide; no effect
+ * until called).  Every wait of a GEMM kernel on a barrier gives up after a time
+ * limit (2 s), records NVFP4_ERR_TIMEOUT in the device status word and lets the
+ * kernel drain its own work and exit, so the context stays usable.
+ *   drop_first_stage != 0: the TMA producer of every CTA skips its first pipeline
+ *     stage, so the waits for that stage run out: the call ends with device
+ *     status NVFP4_ERR_TIMEOUT and unspecified outputs.  0 restores normal work.
+ *   wait_limit_ns > 0 replaces the 2 s limit of each wait; 0 restores it.
+ * Not for use while other GEMM work is in flight. */
+nvfp4_status nvfp4_debug_gemm_fault(int32_t drop_first_stage, uint64_t wait_limit_ns);
+
 /* Human-readable name of a status code (static string). */
 const char* nvfp4_status_string(int32_t status);
 

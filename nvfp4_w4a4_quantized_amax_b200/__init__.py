@@ -68,6 +68,7 @@ EXPORTS = ["nvfp4_version", "nvfp4_status_string", "nvfp4_scales_bytes", "nvfp4_
            "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_cache_bytes", "nvfp4_kv_cache_init",
            "kv_quant_append", "kv_quant_append_noalloc", "kv_dequant_window", "kv_dequant_window_tokens",
            "nvfp4_lora_merge", "nvfp4_amax_history_push", "nvfp4_last_cuda_error_string",
+           "nvfp4_debug_gemm_fault",
            "nvfp4_get_device_status"]
 
 
@@ -86,6 +87,8 @@ def library():
             lib.nvfp4_version.restype = i32
             lib.nvfp4_status_string.restype = ctypes.c_char_p
             lib.nvfp4_status_string.argtypes = [i32]
+            lib.nvfp4_debug_gemm_fault.restype = i32
+            lib.nvfp4_debug_gemm_fault.argtypes = [i32, ctypes.c_uint64]
             lib.nvfp4_last_cuda_error_string.restype = ctypes.c_char_p
             lib.nvfp4_last_cuda_error_string.argtypes = []
             lib.nvfp4_scales_bytes.restype = i32
@@ -308,6 +311,11 @@ def nvfp4_amax_history_push(history, amax_new, gscale_out, stream=None):
     next supplied tensor scale RN(max(history) / 2688) to gscale_out."""
     _check(library().nvfp4_amax_history_push(_ptr(history), history.numel(), _ptr(amax_new), _ptr(gscale_out),
                                              _stream(stream)), "nvfp4_amax_history_push")
+
+
+def debug_gemm_fault(drop_first_stage: bool, wait_limit_ns: int = 0):
+    """Test hook of the GEMM's bounded waits (see nvfp4_debug_gemm_fault)."""
+    _check(library().nvfp4_debug_gemm_fault(1 if drop_first_stage else 0, wait_limit_ns), "nvfp4_debug_gemm_fault")
 
 
 def get_device_status(device: int = 0, clear: bool = False) -> int:

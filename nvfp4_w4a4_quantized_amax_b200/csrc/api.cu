@@ -408,6 +408,11 @@ nvfp4_status nvfp4_amax_history_push(float* history, int32_t len, const float* a
                                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_debug_gemm_fault(int32_t drop_first_stage, uint64_t wait_limit_ns) {
+  nvfp4::gemm_debug_fault(drop_first_stage, (unsigned long long)wait_limit_ns);
+  return NVFP4_OK;
+}
+
 nvfp4_status nvfp4_get_device_status(int32_t device, int32_t* status_out, int32_t clear) {
   if (!status_out) return NVFP4_ERR_INVALID_ARG;
   int prev = 0;

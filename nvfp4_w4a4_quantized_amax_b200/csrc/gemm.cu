@@ -31,6 +31,7 @@
 // asynchronous work (bounded again) before it frees tensor memory and exits.
 #include <cuda.h>
 
+#include <atomic>
 #include <cstring>
 
 #include "common.cuh"
@@ -65,6 +66,10 @@ constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 /*barrie
 
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
+// Test hook for the bounded waits (set only by nvfp4_debug_gemm_fault).
+std::atomic<unsigned long long> g_debug_wait_limit_ns{0};
+std::atomic<int> g_debug_drop_first_stage{0};
+
 struct Params {
   int64_t M, N, K;
   int64_t num_m, num_n, num_k64;  // tiles along M, N and 64-value groups along K
@@ -89,6 +94,7 @@ struct Params {
   float* h_out;
   unsigned* status;
   unsigned long long wait_limit_ns;
+  int drop_first_stage;  // test hook: skip the first stage's loads (the waits for it run out)
 };
 
 // ----------------------------------------------------------------- PTX helpers
@@ -340,6 +346,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          if (p.drop_first_stage && it == 0) continue;  // its full barrier never completes
           const int64_t g0 = ks * 4;
           const int nvalid = (int)min((int64_t)4, p.num_k64 - g0);
           uint8_t* st = smem + s * kStageBytes;
@@ -711,6 +718,7 @@ struct Params2 {
   float* h_out;
   unsigned* status;
   unsigned long long wait_limit_ns;
+  int drop_first_stage;  // test hook: skip the first stage's loads (the waits for it run out)
 };
 
 // 22 warps: six share one of the SM's four 16K-register files, so at most
@@ -788,6 +796,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
+          if (p.drop_first_stage && it == 0) continue;  // its full barrier never completes
           const int64_t g0 = ks * 4;
           const int nvalid = (int)min((int64_t)4, p.num_k64 - g0);
           uint8_t* st = smem + s * kStageBytes;
@@ -1183,7 +1192,8 @@ cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s) {
   p.q_amax_out = g.q_amax_out;
   p.h_out = g.h_out;
   p.status = g.status;
-  p.wait_limit_ns = kWaitLimitNs;
+  p.wait_limit_ns = g_debug_wait_limit_ns.load() ? g_debug_wait_limit_ns.load() : kWaitLimitNs;
+  p.drop_first_stage = g_debug_drop_first_stage.load();
 
   CUtensorMap ma, mw, mc;
   if (!make_code_map(&ma, g.a.codes, g.M, g.K / 2, g.a.ld_codes, 128)) return cudaErrorInvalidValue;
@@ -1265,7 +1275,8 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
   p.q_amax_out = g.q_amax_out;
   p.h_out = g.h_out;
   p.status = g.status;
-  p.wait_limit_ns = kWaitLimitNs;
+  p.wait_limit_ns = g_debug_wait_limit_ns.load() ? g_debug_wait_limit_ns.load() : kWaitLimitNs;
+  p.drop_first_stage = g_debug_drop_first_stage.load();
 
   CUtensorMap ma, mw;
   if (!make_code_map(&ma, g.a.codes, g.M, g.K / 2, g.a.ld_codes, kBM)) return cudaErrorInvalidValue;
@@ -1285,6 +1296,11 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
   const int grid = (int)(p.num_tiles < sms ? p.num_tiles : sms);
   gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mw, mc, p);
   return cudaGetLastError();
+}
+
+void gemm_debug_fault(int drop_first_stage, unsigned long long wait_limit_ns) {
+  g_debug_drop_first_stage.store(drop_first_stage ? 1 : 0);
+  g_debug_wait_limit_ns.store(wait_limit_ns);
 }
 
 }  // namespace nvfp4

@@ -126,5 +126,7 @@ struct GemmArgs {
   unsigned* status;
 };
 cudaError_t launch_gemm(const GemmArgs& a, cudaStream_t s);
+// Test hook of the GEMM's bounded waits (see nvfp4_debug_gemm_fault).
+void gemm_debug_fault(int drop_first_stage, unsigned long long wait_limit_ns);
 
 }  // namespace nvfp4
