@@ -87,6 +87,14 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
+// Programmatic dependent launch: every kernel of the library is launched so that
+// the next one may start before it ends.  pdl_trigger lets the grid launched after
+// this one on the stream begin (its CTAs then wait in pdl_wait); pdl_wait blocks
+// until every grid before this one on the stream has completed and its memory is
+// visible, so it goes before the first read of anything a previous kernel wrote.
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- E2M1
 // Exact E2M1 magnitude index of |x| / D by comparing |x| with each midpoint
 // m * D (m = 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5).  fmaf gives the correctly

@@ -288,6 +288,7 @@ __device__ __forceinline__ float gelu_tanh(float c) {
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w,
                 const __grid_constant__ CUtensorMap map_c, Params p) {
+  pdl_trigger();  // the next kernel on the stream may start its set-up
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + kStages * kStageBytes;  // 1024-aligned
@@ -327,6 +328,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // operands and scales were written by earlier kernels
   const unsigned long long limit = p.wait_limit_ns;
 
   if (warp == 0) {
@@ -729,6 +731,7 @@ template <bool kFused>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     gemm_pair_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_w,
                      const __grid_constant__ CUtensorMap map_c, Params2 p) {
+  pdl_trigger();  // the next kernel on the stream may start its set-up
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* staging = smem + kStages * kStageBytes;
@@ -771,6 +774,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   cluster_sync();  // barriers of both CTAs initialized, tensor memory allocated
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // operands and scales were written by earlier kernels
   const unsigned long long limit = p.wait_limit_ns;
   const int64_t kstages = (p.num_k64 + 3) / 4;
 
@@ -1235,7 +1239,7 @@ cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s) {
   }
   const int64_t max_pairs = resident[dev];
   const int64_t pairs = p.num_tiles < max_pairs ? p.num_tiles : max_pairs;
-  pair::gemm_pair_kernel<kFused><<<(unsigned)(2 * pairs), pair::kThreads, pair::kSmemBytes, s>>>(ma, mw, mc, p);
+  launch_pdl(pair::gemm_pair_kernel<kFused>, (unsigned)(2 * pairs), pair::kThreads, pair::kSmemBytes, s, ma, mw, mc, p);
   return cudaGetLastError();
 }
 
@@ -1294,7 +1298,7 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const int sms = sm_count_gemm();
   const int grid = (int)(p.num_tiles < sms ? p.num_tiles : sms);
-  gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ma, mw, mc, p);
+  launch_pdl(gemm_kernel, grid, kThreads, kSmemBytes, s, ma, mw, mc, p);
   return cudaGetLastError();
 }
 

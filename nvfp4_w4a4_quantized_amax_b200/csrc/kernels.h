@@ -8,6 +8,25 @@
 
 namespace nvfp4 {
 
+// Launch with programmatic stream serialization (the kernel calls pdl_trigger and
+// pdl_wait itself): the launch and the first CTAs of this kernel overlap the tail
+// of the previous kernel on the stream.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, static_cast<Args&&>(args)...);
+}
+
 // CTAs of `kThreads` threads of kernel K that are resident at once on the current
 // device (occupancy x SMs), looked up once per device: grid-stride kernels launch
 // exactly one full wave.

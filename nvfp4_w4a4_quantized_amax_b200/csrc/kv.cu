@@ -71,6 +71,8 @@ struct StatsParams {
 };
 
 __global__ void __launch_bounds__(kStatsThreads) kv_stats_kernel(StatsParams p) {
+  pdl_trigger();
+  pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t c0 = (int64_t)blockIdx.x * kStatsCols + lane * 8;
   const bool active = c0 < p.C;
@@ -250,6 +252,8 @@ struct MuParams {
 // range test every partial sum is an exact double, so the order of the additions
 // does not matter.
 __global__ void __launch_bounds__(kMuThreads) kv_mu_kernel(MuParams p) {
+  pdl_trigger();
+  pdl_wait();
   if (p.sc.words[2]) return;  // non-finite input: the slot stays unchanged
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   constexpr int kWarps = kMuThreads / 32;
@@ -392,6 +396,8 @@ __device__ __forceinline__ void encode_block16(const float (&v)[16], float g, fl
 }
 
 __global__ void __launch_bounds__(kEncThreads) kv_encode_kernel(EncParams p) {
+  pdl_trigger();
+  pdl_wait();
   if (p.words[2]) {  // a NaN or Inf in K or V: report it, leave the slot unchanged
     if (blockIdx.x == 0 && threadIdx.x == 0) set_status(p.status, kStatusNonfinite);
     return;
@@ -462,6 +468,8 @@ struct WindowParams {
 // the output is written at byte 16 hb of k_out / v_out.  A thread tracks the list
 // entry its index falls in and moves on as its index advances.
 __global__ void __launch_bounds__(kEncThreads) kv_window_kernel(WindowParams p) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t total = p.hb_end[p.n_slots - 1];
   const int64_t stride = (int64_t)gridDim.x * kEncThreads;
   int i = -1;
@@ -550,7 +558,7 @@ cudaError_t launch_append_kernels(const KVLayout& L, const void* k, const void* 
   sp.tokens_per_split = (T + nsplits - 1) / nsplits;
   sp.sc = sc;
   dim3 sgrid((unsigned)colblocks, (unsigned)nsplits);
-  kv_stats_kernel<<<sgrid, kStatsThreads, 0, s>>>(sp);
+  launch_pdl(kv_stats_kernel, sgrid, kStatsThreads, 0, s, sp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   MuParams mp;
@@ -563,7 +571,7 @@ cudaError_t launch_append_kernels(const KVLayout& L, const void* k, const void* 
   int lg = 0;
   while ((1ll << lg) < T) ++lg;
   mp.log2T_ceil = lg;
-  kv_mu_kernel<<<(unsigned)((C + kMuCols - 1) / kMuCols), kMuThreads, 0, s>>>(mp);
+  launch_pdl(kv_mu_kernel, (unsigned)((C + kMuCols - 1) / kMuCols), kMuThreads, 0, s, mp);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   EncParams ep;
   ep.k = (const uint8_t*)k;
@@ -580,7 +588,7 @@ cudaError_t launch_append_kernels(const KVLayout& L, const void* k, const void* 
   ep.tokens = (int32_t)T;
   ep.words = sc.words;
   ep.status = status;
-  kv_encode_kernel<<<wave_grid<kv_encode_kernel>(kEncThreads, ep.nblocks), kEncThreads, 0, s>>>(ep);
+  launch_pdl(kv_encode_kernel, wave_grid<kv_encode_kernel>(kEncThreads, ep.nblocks), kEncThreads, 0, s, ep);
   return cudaGetLastError();
 }
 
@@ -629,7 +637,7 @@ cudaError_t launch_kv_window(const KVLayout& L, const int32_t* slots, const int3
   p.v_out = static_cast<uint8_t*>(v_out);
   p.status = status;
   const int grid = wave_grid<kv_window_kernel>(kEncThreads, acc);
-  kv_window_kernel<<<grid, kEncThreads, 0, s>>>(p);
+  launch_pdl(kv_window_kernel, grid, kEncThreads, 0, s, p);
   return cudaGetLastError();
 }
 

@@ -33,6 +33,8 @@ struct LoraParams {
 };
 
 __global__ void __launch_bounds__(kThreads) lora_merge_kernel(LoraParams p) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ __align__(16) float bs[kStep][kRows];  // bs[j][row]
   __shared__ float as[kStep][kCols];
   const int64_t r0 = (int64_t)blockIdx.y * kRows, c0 = (int64_t)blockIdx.x * kCols;
@@ -92,7 +94,7 @@ cudaError_t launch_lora_merge(const LoraArgs& a, cudaStream_t s) {
   p.out = a.out;
   p.ldo = a.ldo;
   dim3 grid((unsigned)((a.cols + kCols - 1) / kCols), (unsigned)((a.rows + kRows - 1) / kRows));
-  lora_merge_kernel<<<grid, kThreads, 0, s>>>(p);
+  launch_pdl(lora_merge_kernel, grid, kThreads, 0, s, p);
   return cudaGetLastError();
 }
 

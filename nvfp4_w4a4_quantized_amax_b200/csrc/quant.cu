@@ -37,6 +37,8 @@ template <bool kBf16>
 __global__ void __launch_bounds__(kThreads) amax_kernel(const uint8_t* __restrict__ x,
                                                         int64_t row_bytes, int64_t nchunks,
                                                         FastDiv cpr, unsigned* amax_bits) {
+  pdl_trigger();
+  pdl_wait();
   unsigned m = 0;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < nchunks; i += stride) {
@@ -80,6 +82,8 @@ struct EncodeParams {
 // One thread encodes one 16-value block: block amax -> E4M3 scale -> 16 codes.
 template <bool kBf16, bool kMma>
 __global__ void __launch_bounds__(kThreads) encode_kernel(EncodeParams p) {
+  pdl_trigger();
+  pdl_wait();
   float g;
   if (p.gscale_in) {
     g = *p.gscale_in;
@@ -179,6 +183,8 @@ struct DequantParams {
 // warp reads 128 contiguous bytes of codes and writes 512 contiguous bytes of bf16.
 template <bool kMma, bool kBf16Out>
 __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantParams p) {
+  pdl_trigger();
+  pdl_wait();
   const float g = *p.gscale;
   const int64_t total = 2 * p.nblocks;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
@@ -217,6 +223,8 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantParams p) {
 constexpr int kHistThreads = 256;
 __global__ void __launch_bounds__(kHistThreads) amax_history_kernel(float* history, int len, const float* amax_new,
                                                                    float* g_out, unsigned* status) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float old[kMaxHistory];
   __shared__ unsigned red[kHistThreads / 32];
   const float a = *amax_new;
@@ -262,10 +270,10 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
     const int64_t cpr = a.cols * esz / 16;
     const int64_t n = a.rows * cpr;
     if (a.x_bf16)
-      amax_kernel<true><<<wave_grid<amax_kernel<true>>(kThreads, n), kThreads, 0, s>>>((const uint8_t*)a.x, a.ldx * esz, n,
+      launch_pdl(amax_kernel<true>, wave_grid<amax_kernel<true>>(kThreads, n), kThreads, 0, s, (const uint8_t*)a.x, a.ldx * esz, n,
                                                          FastDiv((uint32_t)cpr), amax_bits);
     else
-      amax_kernel<false><<<wave_grid<amax_kernel<false>>(kThreads, n), kThreads, 0, s>>>((const uint8_t*)a.x, a.ldx * esz, n,
+      launch_pdl(amax_kernel<false>, wave_grid<amax_kernel<false>>(kThreads, n), kThreads, 0, s, (const uint8_t*)a.x, a.ldx * esz, n,
                                                           FastDiv((uint32_t)cpr), amax_bits);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
@@ -291,11 +299,11 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
   p.status = a.status;
   const int64_t n = p.nvblocks;
   if (a.x_bf16) {
-    if (a.sf_mma) encode_kernel<true, true><<<wave_grid<encode_kernel<true, true>>(kThreads, n), kThreads, 0, s>>>(p);
-    else encode_kernel<true, false><<<wave_grid<encode_kernel<true, false>>(kThreads, n), kThreads, 0, s>>>(p);
+    if (a.sf_mma) launch_pdl(encode_kernel<true, true>, wave_grid<encode_kernel<true, true>>(kThreads, n), kThreads, 0, s, p);
+    else launch_pdl(encode_kernel<true, false>, wave_grid<encode_kernel<true, false>>(kThreads, n), kThreads, 0, s, p);
   } else {
-    if (a.sf_mma) encode_kernel<false, true><<<wave_grid<encode_kernel<false, true>>(kThreads, n), kThreads, 0, s>>>(p);
-    else encode_kernel<false, false><<<wave_grid<encode_kernel<false, false>>(kThreads, n), kThreads, 0, s>>>(p);
+    if (a.sf_mma) launch_pdl(encode_kernel<false, true>, wave_grid<encode_kernel<false, true>>(kThreads, n), kThreads, 0, s, p);
+    else launch_pdl(encode_kernel<false, false>, wave_grid<encode_kernel<false, false>>(kThreads, n), kThreads, 0, s, p);
   }
   return cudaGetLastError();
 }
@@ -316,11 +324,11 @@ cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t s) {
   p.y_row_bytes = a.ldy * (a.y_bf16 ? 2 : 4);
   const int64_t n = 2 * p.nblocks;
   if (a.sf_mma) {
-    if (a.y_bf16) dequant_kernel<true, true><<<wave_grid<dequant_kernel<true, true>>(kThreads, n), kThreads, 0, s>>>(p);
-    else dequant_kernel<true, false><<<wave_grid<dequant_kernel<true, false>>(kThreads, n), kThreads, 0, s>>>(p);
+    if (a.y_bf16) launch_pdl(dequant_kernel<true, true>, wave_grid<dequant_kernel<true, true>>(kThreads, n), kThreads, 0, s, p);
+    else launch_pdl(dequant_kernel<true, false>, wave_grid<dequant_kernel<true, false>>(kThreads, n), kThreads, 0, s, p);
   } else {
-    if (a.y_bf16) dequant_kernel<false, true><<<wave_grid<dequant_kernel<false, true>>(kThreads, n), kThreads, 0, s>>>(p);
-    else dequant_kernel<false, false><<<wave_grid<dequant_kernel<false, false>>(kThreads, n), kThreads, 0, s>>>(p);
+    if (a.y_bf16) launch_pdl(dequant_kernel<false, true>, wave_grid<dequant_kernel<false, true>>(kThreads, n), kThreads, 0, s, p);
+    else launch_pdl(dequant_kernel<false, false>, wave_grid<dequant_kernel<false, false>>(kThreads, n), kThreads, 0, s, p);
   }
   return cudaGetLastError();
 }
@@ -330,7 +338,7 @@ cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t s) {
 namespace nvfp4 {
 cudaError_t launch_amax_history(float* history, int len, const float* amax_new, float* g_out, unsigned* status,
                                 cudaStream_t s) {
-  amax_history_kernel<<<1, kHistThreads, 0, s>>>(history, len, amax_new, g_out, status);
+  launch_pdl(amax_history_kernel, 1, kHistThreads, 0, s, history, len, amax_new, g_out, status);
   return cudaGetLastError();
 }
 }  // namespace nvfp4
