@@ -237,22 +237,22 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     def step(events=None, inputs=None):
         X2, A3, A3B, X5, KVK, KVV = inputs if inputs is not None else (
             x2, a3, a3b, x5, kvd[slot_counter[0] % 2][0], kvd[slot_counter[0] % 2][1])
-        timed("quantize_32768x3072", lambda: nv.nvfp4_quantize(X2, qx2, amax_out=amax[0:1]), 2, events)
+        timed("quantize_32768x3072", lambda: nv.nvfp4_quantize(X2, qx2, amax_out=amax[0:1]), 3, events)
         timed("dequantize_32768x3072", lambda: nv.nvfp4_dequantize(qx2, y2), 1, events)
-        timed("quantize_8192x3072", lambda: nv.nvfp4_quantize(A3, qa3, amax_out=amax[1:2]), 2, events)
-        timed("quantize_8192x14336", lambda: nv.nvfp4_quantize(A3B, qa3b, amax_out=amax[2:3]), 2, events)
+        timed("quantize_8192x3072", lambda: nv.nvfp4_quantize(A3, qa3, amax_out=amax[1:2]), 3, events)
+        timed("quantize_8192x14336", lambda: nv.nvfp4_quantize(A3B, qa3b, amax_out=amax[2:3]), 3, events)
         for i, (k, n) in enumerate(BLOCK_GEMMS):
             a = qa3 if k == 3072 else qa3b
             timed(f"gemm_{k}x{n}", lambda a=a, i=i: nv.nvfp4_gemm(a, wq[i], cs[i]), 1, events)
         slot = slot_counter[0] % SLOTS
-        timed("kv_append_8192", lambda: nv.kv_quant_append(cache, KVK, KVV, slot), 3, events)
+        timed("kv_append_8192", lambda: nv.kv_quant_append(cache, KVK, KVV, slot), 4, events)
         win = [(slot - WINDOW + 1 + j) % SLOTS for j in range(WINDOW)]
         timed("kv_window_4x8192", lambda: nv.kv_dequant_window(cache, win, ko, vo), 1, events)
         slot_counter[0] += 1
-        timed("quantize_8192x3072_ffn", lambda: nv.nvfp4_quantize(X5, qx5, amax_out=amax[3:4]), 2, events)
+        timed("quantize_8192x3072_ffn", lambda: nv.nvfp4_quantize(X5, qx5, amax_out=amax[3:4]), 3, events)
         timed("gemm_ffn_up_gelu_requant", lambda: nv.nvfp4_gemm(qx5, q1, None, act=nv.ACT_GELU_TANH,
                                                                 q_out=qh, q_gscale_in=g_h,
-                                                                q_amax_out=amax[6:7]), 1, events)
+                                                                q_amax_out=amax[6:7]), 2, events)
         timed("amax_history_push", lambda: nv.nvfp4_amax_history_push(hist, amax[6:7], g_h), 1, events)
         timed("gemm_ffn_down_bf16", lambda: nv.nvfp4_gemm(qh, q2, y5), 1, events)
 

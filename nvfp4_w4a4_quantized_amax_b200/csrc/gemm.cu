@@ -1205,7 +1205,7 @@ cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s) {
   memset(&mc, 0, sizeof(mc));
   if (g.c && !make_out_map(&mc, g.c, g.M, g.N, g.ldc, g.c_bf16, true)) return cudaErrorInvalidValue;
   if (g.q_amax_out) {
-    cudaError_t e = cudaMemsetAsync(g.q_amax_out, 0, sizeof(float), s);
+    cudaError_t e = launch_zero_words(g.q_amax_out, 1, s);
     if (e != cudaSuccess) return e;
   }
   static bool done[64];
@@ -1290,7 +1290,7 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
   if (g.c && !make_out_map(&mc, g.c, g.M, g.N, g.ldc, g.c_bf16)) return cudaErrorInvalidValue;
 
   if (g.q_amax_out) {
-    cudaError_t e = cudaMemsetAsync(g.q_amax_out, 0, sizeof(float), s);
+    cudaError_t e = launch_zero_words(g.q_amax_out, 1, s);
     if (e != cudaSuccess) return e;
   }
   static bool done[64];

@@ -105,6 +105,9 @@ constexpr int kMaxWindowSlots = 64;
 cudaError_t launch_kv_window(const KVLayout& c, const int32_t* slots, const int32_t* tokens, int32_t n_slots,
                              void* k_out, void* v_out, unsigned* status, cudaStream_t s);
 
+// Zero n_words 32-bit words of device memory (a PDL-launched kernel, not a memset).
+cudaError_t launch_zero_words(void* p, int n_words, cudaStream_t s);
+
 constexpr int kMaxHistory = 1024;
 cudaError_t launch_amax_history(float* history, int len, const float* amax_new, float* g_out, unsigned* status,
                                 cudaStream_t s);

@@ -604,7 +604,7 @@ cudaError_t launch_kv_append(const KVLayout& L, const void* k, const void* v, in
                              unsigned* status, cudaStream_t s) {
   const int64_t C = (int64_t)L.heads * L.head_dim;
   Scratch sc = scratch_at(L.base + L.off_scratch, C);
-  cudaError_t e = cudaMemsetAsync(sc.words, 0, 3 * sizeof(unsigned), s);
+  cudaError_t e = launch_zero_words(sc.words, 3, s);
   if (e != cudaSuccess) return e;
 
   return launch_append_kernels(L, k, v, tokens, slot, sc, status, s);
@@ -686,7 +686,7 @@ cudaError_t launch_kv_append_noalloc(const KVLayout& L, const void* k, const voi
   Scratch sc = scratch_at(scratch, C);
   // the words accumulate with atomics: they must start at zero on every call; the
   // statistics of every split in use are fully rewritten by kv_stats_kernel
-  if ((e = cudaMemsetAsync(sc.words, 0, 3 * sizeof(unsigned), s)) != cudaSuccess) return e;
+  if ((e = launch_zero_words(sc.words, 3, s)) != cudaSuccess) return e;
 
   return launch_append_kernels(L, k, v, tokens, slot, sc, status, s);
 }

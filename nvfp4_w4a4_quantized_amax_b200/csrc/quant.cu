@@ -218,6 +218,14 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantParams p) {
 }
 
 
+// Zeroes n words before an accumulation: a kernel rather than a memset, so that
+// its launch overlaps the previous kernel.  It does not trigger its dependents
+// early: the kernel after it starts only once it is done (as after a memset).
+__global__ void zero_words_kernel(unsigned* p, int n) {
+  pdl_wait();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) p[i] = 0u;
+}
+
 // Amax history of a requantizing epilogue (newest first): shift in *amax_new and
 // write g = RN(max(history) / 2688).  One CTA; a non-finite value changes nothing.
 constexpr int kHistThreads = 256;
@@ -257,7 +265,7 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
   const int64_t nb = a.cols / 16;
   unsigned* amax_bits = reinterpret_cast<unsigned*>(a.amax_out);
   if (a.amax_out) {
-    cudaError_t e = cudaMemsetAsync(a.amax_out, 0, sizeof(float), s);
+    cudaError_t e = launch_zero_words(a.amax_out, 1, s);
     if (e != cudaSuccess) return e;
   }
   if (a.rows == 0) {
@@ -336,6 +344,11 @@ cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t s) {
 }  // namespace nvfp4
 
 namespace nvfp4 {
+cudaError_t launch_zero_words(void* p, int n_words, cudaStream_t s) {
+  launch_pdl(zero_words_kernel, 1, 32, 0, s, static_cast<unsigned*>(p), n_words);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_amax_history(float* history, int len, const float* amax_new, float* g_out, unsigned* status,
                                 cudaStream_t s) {
   launch_pdl(amax_history_kernel, 1, kHistThreads, 0, s, history, len, amax_new, g_out, status);
