@@ -642,7 +642,10 @@ constexpr int kSfaBytes = 4 * 512;                // own 128 rows, 4 groups
 constexpr int kSfbBytes = kWTiles * 4 * 512;      // all kBN W rows of the tile x 4 groups
 constexpr int kStageBytes = kABytes + kBBytes + kSfaBytes + kSfbBytes;
 static_assert(kStageBytes % 1024 == 0, "stages must keep 1024-byte alignment");
-constexpr int kStagingBytesPerWarp = 32 * 64;   // one output box: 32 rows x 64 bytes
+// Output staging: 32 rows x 64 bytes per epilogue warp.  A bf16 output box is one
+// warp's buffer; an FP32 box (128 rows x 16 columns) is the 4 buffers of a column
+// group, contiguous because the group's warps are consecutive.
+constexpr int kStagingBytesPerWarp = 32 * 64;
 constexpr int kStagingBytes = kEpiWarps * kStagingBytesPerWarp;
 constexpr int kSmemBytes = kStages * kStageBytes + kStagingBytes + 1024 + 1024;
 static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
@@ -675,6 +678,18 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t addr, uint32_t rank) {
 // Arrive on a barrier of another CTA of the cluster.  What it orders is tensor
 // memory traffic, which the tcgen05 fences around the arrive and the wait order;
 // no cluster-scope memory fence is needed (and one costs a membar per arrive).
+// AND of `ok` over the 128 threads (4 warps) that use named barrier `id`; every
+// one of them must call it.
+__device__ __forceinline__ bool group_all(uint32_t id, bool ok) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred q, p;\n setp.ne.u32 q, %1, 0;\n bar.red.and.pred p, %2, 128, q;\n selp.u32 %0, 1, 0, p;\n}"
+      : "=r"(r)
+      : "r"((uint32_t)ok), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
   asm volatile("mbarrier.arrive.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr) : "memory");
 }
@@ -952,12 +967,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       if (blockIdx.x == 0 && threadIdx.x == kEpiWarp0 * 32) *p.q_gscale_out = gq;
     }
     const bool has_c = kFused ? p.has_c : true;
+    // FP32 output goes through one 128-row box per column group; the group's 4 warps
+    // synchronise on named barrier 1 + cgroup and so must also leave the tile loop
+    // together.
+    const bool grouped = has_c && !p.c_bf16;
+    const uint32_t gbar = 1u + (uint32_t)cgroup;
+    const uint32_t gbuf = smem_u32(staging) + (uint32_t)(cgroup * 4 * kStagingBytesPerWarp);
     unsigned amax_bits = 0;
     uint32_t tcount = 0;
     for (int64_t tile = pair; tile < p.num_tiles; tile += num_pairs, ++tcount) {
       const int a = tcount % kAccStages;
       const uint32_t aph = (tcount / kAccStages) & 1u;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&tfull_bar[a]), aph, abort_flag, limit))) {
+      bool got = __all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&tfull_bar[a]), aph, abort_flag, limit));
+      if (grouped) got = group_all(gbar, got);
+      if (!got) {
         if (lane == 0) set_status(p.status, kStatusTimeout);
         *abort_flag = 1;
         break;
@@ -1001,20 +1024,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               asm volatile("cp.async.bulk.commit_group;" ::: "memory");
             }
           } else {
-            // FP32: two 32 x 16 boxes through the one staging box
+            // FP32: the group's 4 warps fill one 128 x 16 box (8 KB), one thread stores it
 #pragma unroll
             for (int b = 0; b < 2; ++b) {
-              if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-              __syncwarp();
+              if (quarter == 0 && lane == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+              asm volatile("bar.sync %0, 128;" ::"r"(gbar) : "memory");
+              const int rr = quarter * 32 + lane;
 #pragma unroll
               for (int u = 0; u < 4; ++u)
-                st_shared_v4(buf + lane * 64 + ((u ^ ((lane >> 1) & 3)) * 16),
+                st_shared_v4(gbuf + rr * 64 + ((u ^ ((rr >> 1) & 3)) * 16),
                              make_uint4(__float_as_uint(v[16 * b + 4 * u]), __float_as_uint(v[16 * b + 4 * u + 1]),
                                         __float_as_uint(v[16 * b + 4 * u + 2]), __float_as_uint(v[16 * b + 4 * u + 3])));
               asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-              __syncwarp();
-              if (lane == 0) {
-                tma_store_2d(&map_c, buf, (int32_t)(col0 + 16 * b), out_row);
+              asm volatile("bar.sync %0, 128;" ::"r"(gbar) : "memory");
+              if (quarter == 0 && lane == 0) {
+                tma_store_2d(&map_c, gbuf, (int32_t)(col0 + 16 * b), (int32_t)(mt * kBM + rank * 128));
                 asm volatile("cp.async.bulk.commit_group;" ::: "memory");
               }
             }
@@ -1124,18 +1148,18 @@ bool make_code_map(CUtensorMap* m, const uint8_t* base, int64_t rows, int64_t kb
 }
 
 // 2-D map over the output C [M, N] (row pitch ldc elements) for the epilogue's
-// TMA stores, boxes of 32 rows swizzled like the staging buffers: 32 columns
-// (128 B rows, 128-byte swizzle, FP32; 64 B rows, 64-byte swizzle, bf16), or with
-// `rows64` 64-byte rows for both types (16 FP32 or 32 bf16 columns).
+// TMA stores, boxes of `box_rows` rows swizzled like the staging buffers: 32
+// columns (128 B rows, 128-byte swizzle, FP32; 64 B rows, 64-byte swizzle, bf16),
+// or with `rows64` 64-byte rows for both types (16 FP32 or 32 bf16 columns).
 bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_t ld, bool bf16,
-                  bool rows64 = false) {
+                  bool rows64 = false, uint32_t box_rows = 32) {
   EncodeTiledFn fn = get_encode_fn();
   if (!fn) return false;
   const int64_t esz = bf16 ? 2 : 4;
   const bool sw64 = bf16 || rows64;
   cuuint64_t dims[2] = {(cuuint64_t)cols, (cuuint64_t)rows};
   cuuint64_t strides[1] = {(cuuint64_t)(ld * esz)};
-  cuuint32_t box[2] = {(cuuint32_t)(sw64 ? 64 / esz : 32), 32};
+  cuuint32_t box[2] = {(cuuint32_t)(sw64 ? 64 / esz : 32), box_rows};
   cuuint32_t estr[2] = {1, 1};
   return fn(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, base, dims, strides,
             box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -1203,7 +1227,9 @@ cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s) {
   if (!make_code_map(&ma, g.a.codes, g.M, g.K / 2, g.a.ld_codes, 128)) return cudaErrorInvalidValue;
   if (!make_code_map(&mw, g.w.codes, g.N, g.K / 2, g.w.ld_codes, pair::kBNHalf)) return cudaErrorInvalidValue;
   memset(&mc, 0, sizeof(mc));
-  if (g.c && !make_out_map(&mc, g.c, g.M, g.N, g.ldc, g.c_bf16, true)) return cudaErrorInvalidValue;
+  // FP32 output: one 128-row box per column group of the epilogue (see the kernel)
+  if (g.c && !make_out_map(&mc, g.c, g.M, g.N, g.ldc, g.c_bf16, true, g.c_bf16 ? 32u : 128u))
+    return cudaErrorInvalidValue;
   if (g.q_amax_out) {
     cudaError_t e = launch_zero_words(g.q_amax_out, 1, s);
     if (e != cudaSuccess) return e;
