@@ -261,13 +261,10 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       : "memory");
 }
 
-__device__ __forceinline__ void tmem_st_32x32b_x16(uint32_t taddr, const uint32_t (&r)[16]) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
-      "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
+__device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
+  asm volatile("tcgen05.st.sync.aligned.32x32b.x4.b32 [%0], {%1,%2,%3,%4};" ::"r"(taddr), "r"(v.x), "r"(v.y),
+               "r"(v.z), "r"(v.w)
+               : "memory");
 }
 
 // GELU, tanh form: 0.5 c (1 + tanh(u)) with u = sqrt(2/pi) (c + 0.044715 c^3),
@@ -632,10 +629,29 @@ constexpr int kWTiles = kBN / 128;  // 128-row W scale tiles per pair tile
 constexpr int kStages = 5;
 constexpr int kSfSlots = kStages;  // one per pipeline stage
 constexpr int kAccStages = kBN == 256 ? 1 : 2;
-constexpr int kEpiWarps = 16;  // 4 per tensor-memory lane quarter, 64 columns each
-constexpr int kEpiWarp0 = 2;
-constexpr int kSfWarp0 = kEpiWarp0 + kEpiWarps;
-constexpr int kThreads = 32 * (2 + kEpiWarps + 4);
+// Warp roles, in 4-warp groups (the unit of register reallocation):
+//   warpgroup 0  warp 0 TMA producer, warp 1 MMA issuer (leader CTA), warps 2-3 idle
+//   warpgroup 1  warps 4..7 scale factors, one per tensor-memory lane quarter
+//   2..5         warps 8..23 epilogue, 4 per lane quarter, 64 columns each
+constexpr int kEpiWarps = 16;
+constexpr int kSfWarp0 = 4;
+constexpr int kEpiWarp0 = 8;
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);  // 768
+// Registers: the kernel is launched with kRegsLaunch a thread (24 warps, six on each
+// of the SM's four 16K-register files: 16384 / 192 = 85, allocated in steps of 8).
+// Warpgroups 0 and 1 then release registers with setmaxnreg.dec and the four
+// epilogue warpgroups take them with setmaxnreg.inc; an increase waits until the
+// released registers cover it, so the split must balance exactly (the host checks
+// the compiled launch count before the first launch).
+constexpr int kRegsLaunch = 80;
+constexpr int kRegsCtl = 40;   // warpgroup 0 (fewer make the MMA loop spill)
+constexpr int kRegsSf = 24;    // warpgroup 1
+constexpr int kRegsEpi = 104;  // warpgroups 2..5: 64 accumulator values a thread + work
+static_assert(4 * (kRegsEpi - kRegsLaunch) <= (kRegsLaunch - kRegsCtl) + (kRegsLaunch - kRegsSf),
+              "the epilogue's extra registers must come from warpgroups 0 and 1");
+static_assert(kRegsCtl % 8 == 0 && kRegsSf % 8 == 0 && kRegsEpi % 8 == 0 && kRegsCtl >= 24 && kRegsSf >= 24 &&
+                  kRegsCtl <= kRegsLaunch && kRegsSf <= kRegsLaunch && kRegsEpi >= kRegsLaunch,
+              "setmaxnreg counts");
 constexpr int kABytes = 128 * kBKBytes;           // 16 KB
 constexpr int kBBytes = kBNHalf * kBKBytes;       // 8 or 16 KB
 constexpr int kSfaBytes = 4 * 512;                // own 128 rows, 4 groups
@@ -662,6 +678,15 @@ __device__ __forceinline__ uint32_t cluster_rank() {
   uint32_t r;
   asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
   return r;
+}
+
+template <int kRegs>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <int kRegs>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
 }
 
 __device__ __forceinline__ void cluster_sync() {
@@ -738,8 +763,6 @@ struct Params2 {
   int drop_first_stage;  // test hook: skip the first stage's loads (the waits for it run out)
 };
 
-// 22 warps: six share one of the SM's four 16K-register files, so at most
-// 16384 / (6 * 32) = 85 registers a thread (80 after allocation rounding).
 // kFused = false: plain FP32/bf16 output.  kFused = true: the general epilogue
 // (GELU, h_out, max|h|, NVFP4 requantization, optional C).
 template <bool kFused>
@@ -793,106 +816,111 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
   const unsigned long long limit = p.wait_limit_ns;
   const int64_t kstages = (p.num_k64 + 3) / 4;
 
-  if (warp == 0) {
-    // ------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
-      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
-      uint32_t it = 0;
-      bool ok = true;
-      for (int64_t tile = pair; tile < p.num_tiles && ok; tile += num_pairs) {
-        const int64_t mt = tile % p.num_m, nt = tile / p.num_m;
-        const int64_t a_rt = mt * 2 + rank;                 // this CTA's 128-row tile of A
-        const bool has_sfa = a_rt < p.a_row_tiles;
-        const int64_t n0 = nt * kBN;
-        const int64_t w_rt = n0 / 128;  // first 128-row W scale tile of the pair tile
-        int w_tiles = 0;                // W scale tiles present (the last pair tile may be ragged)
-        for (int t = 0; t < kWTiles; ++t) w_tiles += (w_rt + t < p.w_row_tiles) ? 1 : 0;
-        for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1u;
-          if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag, limit)) {
-            ok = false;
-            break;
+  if (warp < kSfWarp0) {
+    // warpgroup 0: producer (warp 0), MMA issuer (warp 1); warps 2 and 3 idle
+    regs_dec<kRegsCtl>();
+    if (warp == 0) {
+      // ------------------------------------------------------------ producer (both CTAs)
+      if (lane == 0) {
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+        asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_w)) : "memory");
+        uint32_t it = 0;
+        bool ok = true;
+        for (int64_t tile = pair; tile < p.num_tiles && ok; tile += num_pairs) {
+          const int64_t mt = tile % p.num_m, nt = tile / p.num_m;
+          const int64_t a_rt = mt * 2 + rank;                 // this CTA's 128-row tile of A
+          const bool has_sfa = a_rt < p.a_row_tiles;
+          const int64_t n0 = nt * kBN;
+          const int64_t w_rt = n0 / 128;  // first 128-row W scale tile of the pair tile
+          int w_tiles = 0;                // W scale tiles present (the last pair tile may be ragged)
+          for (int t = 0; t < kWTiles; ++t) w_tiles += (w_rt + t < p.w_row_tiles) ? 1 : 0;
+          for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
+            const int s = it % kStages;
+            const uint32_t ph = (it / kStages) & 1u;
+            if (!mbar_wait(smem_u32(&empty_bar[s]), ph ^ 1u, abort_flag, limit)) {
+              ok = false;
+              break;
+            }
+            if (p.drop_first_stage && it == 0) continue;  // its full barrier never completes
+            const int64_t g0 = ks * 4;
+            const int nvalid = (int)min((int64_t)4, p.num_k64 - g0);
+            uint8_t* st = smem + s * kStageBytes;
+            const uint32_t fb = smem_u32(&full_bar[s]);
+            const uint32_t bytes = kABytes + kBBytes + (has_sfa ? nvalid * 512 : 0) + w_tiles * nvalid * 512;
+            mbar_arrive_expect_tx(fb, bytes);
+            tma_load_2d(smem_u32(st), &map_a, fb, (int32_t)(ks * kBKBytes), (int32_t)(mt * kBM + rank * 128));
+            tma_load_2d(smem_u32(st + kABytes), &map_w, fb, (int32_t)(ks * kBKBytes),
+                        (int32_t)(n0 + rank * kBNHalf));
+            if (has_sfa)
+              bulk_load(smem_u32(st + kABytes + kBBytes), p.sfa + a_rt * p.sf_row_tile_bytes + g0 * 512,
+                        nvalid * 512, fb);
+            for (int t = 0; t < w_tiles; ++t)
+              bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes + t * 2048),
+                        p.sfw + (w_rt + t) * p.sf_row_tile_bytes + g0 * 512, nvalid * 512, fb);
           }
-          if (p.drop_first_stage && it == 0) continue;  // its full barrier never completes
-          const int64_t g0 = ks * 4;
-          const int nvalid = (int)min((int64_t)4, p.num_k64 - g0);
-          uint8_t* st = smem + s * kStageBytes;
-          const uint32_t fb = smem_u32(&full_bar[s]);
-          const uint32_t bytes = kABytes + kBBytes + (has_sfa ? nvalid * 512 : 0) + w_tiles * nvalid * 512;
-          mbar_arrive_expect_tx(fb, bytes);
-          tma_load_2d(smem_u32(st), &map_a, fb, (int32_t)(ks * kBKBytes), (int32_t)(mt * kBM + rank * 128));
-          tma_load_2d(smem_u32(st + kABytes), &map_w, fb, (int32_t)(ks * kBKBytes),
-                      (int32_t)(n0 + rank * kBNHalf));
-          if (has_sfa)
-            bulk_load(smem_u32(st + kABytes + kBBytes), p.sfa + a_rt * p.sf_row_tile_bytes + g0 * 512,
-                      nvalid * 512, fb);
-          for (int t = 0; t < w_tiles; ++t)
-            bulk_load(smem_u32(st + kABytes + kBBytes + kSfaBytes + t * 2048),
-                      p.sfw + (w_rt + t) * p.sf_row_tile_bytes + g0 * 512, nvalid * 512, fb);
         }
-      }
-      if (!ok) {
-        set_status(p.status, kStatusTimeout);
-        *abort_flag = 1;
-      }
-      const uint32_t n_issued = it;
-      for (uint32_t j = (n_issued > (uint32_t)kStages ? n_issued - kStages : 0); j < n_issued; ++j)
-        mbar_wait_drain(smem_u32(&full_bar[j % kStages]), (j / kStages) & 1u, limit);
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer (leader CTA)
-    if (leader && lane == 0) {
-      uint32_t it = 0, tcount = 0;
-      bool ok = true;
-      for (int64_t tile = pair; tile < p.num_tiles && ok; tile += num_pairs, ++tcount) {
-        const int a = tcount % kAccStages;
-        const uint32_t aph = (tcount / kAccStages) & 1u;
-        if (!mbar_wait(smem_u32(&tempty_bar[a]), aph ^ 1u, abort_flag, limit)) {
-          ok = false;
-          break;
+        if (!ok) {
+          set_status(p.status, kStatusTimeout);
+          *abort_flag = 1;
         }
-        tc_fence_after();
-        const uint32_t d_tmem = tmem_base + a * kBN;
-        for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
-          const int s = it % kStages;
-          const uint32_t ph = (it / kStages) & 1u;
-          if (!mbar_wait(smem_u32(&sf_bar[s]), ph, abort_flag, limit)) {
+        const uint32_t n_issued = it;
+        for (uint32_t j = (n_issued > (uint32_t)kStages ? n_issued - kStages : 0); j < n_issued; ++j)
+          mbar_wait_drain(smem_u32(&full_bar[j % kStages]), (j / kStages) & 1u, limit);
+      }
+    } else if (warp == 1) {
+      // ------------------------------------------------------------ MMA issuer (leader CTA)
+      if (leader && lane == 0) {
+        uint32_t it = 0, tcount = 0;
+        bool ok = true;
+        for (int64_t tile = pair; tile < p.num_tiles && ok; tile += num_pairs, ++tcount) {
+          const int a = tcount % kAccStages;
+          const uint32_t aph = (tcount / kAccStages) & 1u;
+          if (!mbar_wait(smem_u32(&tempty_bar[a]), aph ^ 1u, abort_flag, limit)) {
             ok = false;
             break;
           }
           tc_fence_after();
-          const int nvalid = (int)min((int64_t)4, p.num_k64 - ks * 4);
-          uint8_t* st = smem + s * kStageBytes;
-          const uint32_t a_addr = smem_u32(st), b_addr = smem_u32(st + kABytes);
-          const uint32_t sf_slot = tmem_base + kSfColBase + s * kSfSlotCols;
-          // descriptors of MMA k: start address + 32 k bytes, i.e. + 2 k in the
-          // 16-byte address field (stage addresses stay far below its 2^18 bytes)
-          const uint64_t ad0 = smem_desc(a_addr, 16, 1024, 2), bd0 = smem_desc(b_addr, 16, 1024, 2);
-          if (nvalid == 4) {
-#pragma unroll
-            for (int k = 0; k < 4; ++k)
-              mma2(d_tmem, ad0 + 2 * k, bd0 + 2 * k, sf_slot + k * kSfPerMma, sf_slot + k * kSfPerMma + 4,
-                   (ks > 0 || k > 0) ? 1u : 0u);
-          } else {
-            for (int k = 0; k < nvalid; ++k)
-              mma2(d_tmem, ad0 + 2 * k, bd0 + 2 * k, sf_slot + k * kSfPerMma, sf_slot + k * kSfPerMma + 4,
-                   (ks > 0 || k > 0) ? 1u : 0u);
+          const uint32_t d_tmem = tmem_base + a * kBN;
+          for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
+            const int s = it % kStages;
+            const uint32_t ph = (it / kStages) & 1u;
+            if (!mbar_wait(smem_u32(&sf_bar[s]), ph, abort_flag, limit)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const int nvalid = (int)min((int64_t)4, p.num_k64 - ks * 4);
+            uint8_t* st = smem + s * kStageBytes;
+            const uint32_t a_addr = smem_u32(st), b_addr = smem_u32(st + kABytes);
+            const uint32_t sf_slot = tmem_base + kSfColBase + s * kSfSlotCols;
+            // descriptors of MMA k: start address + 32 k bytes, i.e. + 2 k in the
+            // 16-byte address field (stage addresses stay far below its 2^18 bytes)
+            const uint64_t ad0 = smem_desc(a_addr, 16, 1024, 2), bd0 = smem_desc(b_addr, 16, 1024, 2);
+            if (nvalid == 4) {
+  #pragma unroll
+              for (int k = 0; k < 4; ++k)
+                mma2(d_tmem, ad0 + 2 * k, bd0 + 2 * k, sf_slot + k * kSfPerMma, sf_slot + k * kSfPerMma + 4,
+                     (ks > 0 || k > 0) ? 1u : 0u);
+            } else {
+              for (int k = 0; k < nvalid; ++k)
+                mma2(d_tmem, ad0 + 2 * k, bd0 + 2 * k, sf_slot + k * kSfPerMma, sf_slot + k * kSfPerMma + 4,
+                     (ks > 0 || k > 0) ? 1u : 0u);
+            }
+            commit2(smem_u32(&empty_bar[s]), (uint16_t)0x3);
           }
-          commit2(smem_u32(&empty_bar[s]), (uint16_t)0x3);
+          if (!ok) break;
+          commit2(smem_u32(&tfull_bar[a]), (uint16_t)0x3);
         }
-        if (!ok) break;
-        commit2(smem_u32(&tfull_bar[a]), (uint16_t)0x3);
+        if (!ok) {
+          set_status(p.status, kStatusTimeout);
+          *abort_flag = 1;
+        }
+        commit2(smem_u32(done_bar), (uint16_t)0x1);
+        mbar_wait_drain(smem_u32(done_bar), 0, limit);
       }
-      if (!ok) {
-        set_status(p.status, kStatusTimeout);
-        *abort_flag = 1;
-      }
-      commit2(smem_u32(done_bar), (uint16_t)0x1);
-      mbar_wait_drain(smem_u32(done_bar), 0, limit);
     }
-  } else if (warp >= kSfWarp0) {
+  } else if (warp < kEpiWarp0) {
+    regs_dec<kRegsSf>();
     // ------------------------------------------------------------ scale factors (both CTAs)
     // Slot of stage s, MMA k (c = kSfPerMma k): columns c + 0..3 hold this CTA's A
     // scales (lane l, column j: rows l + 32 j of its 128 rows), c + 4 .. c + 4 +
@@ -918,25 +946,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         const int nvalid = (int)min((int64_t)4, p.num_k64 - ks * 4);
         const uint8_t* sfa = smem + s * kStageBytes + kABytes + kBBytes;
         const uint8_t* sfb = sfa + kSfaBytes;
-        uint32_t r[kSfSlotCols];
+        const uint32_t slot = tmem_base + ((uint32_t)(quarter * 32) << 16) + kSfColBase + s * kSfSlotCols;
 #pragma unroll
         for (int k = 0; k < 4; ++k) {
           uint4 a = make_uint4(0, 0, 0, 0);
           if (k < nvalid && has_sfa) a = *reinterpret_cast<const uint4*>(sfa + k * 512 + lane * 16);
-          r[kSfPerMma * k + 0] = a.x; r[kSfPerMma * k + 1] = a.y;
-          r[kSfPerMma * k + 2] = a.z; r[kSfPerMma * k + 3] = a.w;
+          tmem_st_32x32b_x4(slot + kSfPerMma * k, a);
 #pragma unroll
           for (int t = 0; t < kWTiles; ++t) {
             uint4 b = make_uint4(0, 0, 0, 0);
             if (k < nvalid && w_rt + t < p.w_row_tiles)
               b = *reinterpret_cast<const uint4*>(sfb + t * 2048 + k * 512 + lane * 16);
-            r[kSfPerMma * k + 4 + 4 * t] = b.x; r[kSfPerMma * k + 5 + 4 * t] = b.y;
-            r[kSfPerMma * k + 6 + 4 * t] = b.z; r[kSfPerMma * k + 7 + 4 * t] = b.w;
+            tmem_st_32x32b_x4(slot + kSfPerMma * k + 4 + 4 * t, b);
           }
         }
-        const uint32_t slot = tmem_base + ((uint32_t)(quarter * 32) << 16) + kSfColBase + s * kSfSlotCols;
-        tmem_st_32x32b_x32(slot, *reinterpret_cast<const uint32_t(*)[32]>(&r[0]));
-        if constexpr (kSfSlotCols == 48) tmem_st_32x32b_x16(slot + 32, *reinterpret_cast<const uint32_t(*)[16]>(&r[32]));
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
         tc_fence_before();
         __syncwarp();
@@ -948,6 +971,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
       *abort_flag = 1;
     }
   } else {
+    regs_inc<kRegsEpi>();
     // ------------------------------------------------------------ epilogue (both CTAs)
     // Warp w reads tensor-memory lane quarter w % 4 (rows 32 (w % 4) .. + 31 of this
     // CTA's 128) and columns [64 g, 64 g + 64), g = (w - kEpiWarp0) / 4.  It takes
@@ -1245,6 +1269,13 @@ cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
   if (resident[dev] == 0) {
+    // The kernel's register split (setmaxnreg) balances only for this launch count:
+    // with fewer registers at launch its epilogue warps would wait for registers
+    // that are never released.
+    cudaFuncAttributes fa;
+    e = cudaFuncGetAttributes(&fa, pair::gemm_pair_kernel<kFused>);
+    if (e != cudaSuccess) return e;
+    if (fa.numRegs != pair::kRegsLaunch) return cudaErrorInvalidKernelImage;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(2 * (sm_count_gemm() / 2)), 1, 1);
     cfg.blockDim = dim3(pair::kThreads, 1, 1);
