@@ -140,7 +140,11 @@ typedef enum { NVFP4_ACT_NONE = 0, NVFP4_ACT_GELU_TANH = 1 } nvfp4_activation;
  *                 GEMM ends, so it is SUPPLIED:
  *   q_gscale_in : device FP32 g used for q_out (required with q_out; copied to
  *                 *q_out->gscale).
- *   q_amax_out  : device FP32, nullable: receives max|h| (calibrates the next call).
+ *                 Non-finite h: a 16-block holding a NaN gets the E4M3 NaN scale
+ *                 (0x7F) and codes that keep only the signs; a block with +-inf and
+ *                 no NaN saturates (scale 448, code +-6 for the infinities).
+ *   q_amax_out  : device FP32, nullable: receives max|h| (calibrates the next call);
+ *                 NaN when h holds a NaN, so an amax history push rejects it.
  *   h_out       : device FP32 [M, N] (ld = N), nullable: also store h (verification).
  */
 typedef struct nvfp4_epilogue {

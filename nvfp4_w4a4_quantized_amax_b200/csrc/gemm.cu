@@ -269,6 +269,13 @@ __device__ __forceinline__ void tmem_st_32x32b_x4(uint32_t taddr, uint4 v) {
                : "memory");
 }
 
+// max(a, b) that returns NaN when either operand is NaN
+__device__ __forceinline__ float fmax_nan(float a, float b) {
+  float r;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+  return r;
+}
+
 // GELU, tanh form: 0.5 c (1 + tanh(u)) with u = sqrt(2/pi) (c + 0.044715 c^3),
 // evaluated through the identity 0.5 (1 + tanh(u)) = 1 / (1 + exp(-2u)):
 //   h = c / (1 + 2^x),  x = -2 u log2(e) = c (A c^2 + B),
@@ -558,7 +565,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               if (i < nvc) hd[i] = v[i];
           }
         }
-        if (p.q_amax_out) {
+        if (p.q_amax_out && !p.q_codes) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (i < nvc) amax_bits = max(amax_bits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
@@ -569,9 +576,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
             float s0[8], s1[8];
+            // block max of |h|, NaN-propagating: a NaN makes the block's scale the
+            // E4M3 NaN and (above +inf as bits) max|h| for q_amax_out non-finite
             float amax_b = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(v[16 * b + k]));
+            for (int k = 0; k < 16; ++k) amax_b = fmax_nan(amax_b, fabsf(v[16 * b + k]));
+            amax_bits = max(amax_bits, __float_as_uint(amax_b));
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               s0[k] = v[16 * b + k];
@@ -1092,7 +1102,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               if (i < nvc) hd[i] = v[i];
           }
         }
-        if (p.q_amax_out) {
+        if (p.q_amax_out && !p.q_codes) {
 #pragma unroll
           for (int i = 0; i < 32; ++i)
             if (i < nvc) amax_bits = max(amax_bits, __float_as_uint(v[i]) & 0x7FFFFFFFu);
@@ -1103,9 +1113,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int b = 0; b < 2; ++b) {
             float s0[8], s1[8];
+            // block max of |h|, NaN-propagating: a NaN makes the block's scale the
+            // E4M3 NaN and (above +inf as bits) max|h| for q_amax_out non-finite
             float amax_b = 0.0f;
 #pragma unroll
-            for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(v[16 * b + k]));
+            for (int k = 0; k < 16; ++k) amax_b = fmax_nan(amax_b, fabsf(v[16 * b + k]));
+            amax_bits = max(amax_bits, __float_as_uint(amax_b));
 #pragma unroll
             for (int k = 0; k < 8; ++k) {
               s0[k] = v[16 * b + k];

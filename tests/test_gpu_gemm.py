@@ -77,6 +77,56 @@ def test_zero_rows_and_columns_are_exact(cuda_dev):
     assert_within_bound(got, ref, bound)
 
 
+@pytest.mark.parametrize("M,N", [(256, 512), (128, 256)])  # CTA-pair kernel, single-CTA kernel
+def test_fused_epilogue_nonfinite_blocks(cuda_dev, M, N):
+    """A tensor scale of A large enough to overflow part of c: GELU(+inf) = +inf and
+    GELU(-inf) = -inf * 0 = NaN.  A 16-block of h holding a NaN gets the E4M3 NaN scale
+    0x7F and codes that keep only the signs; a block with infinities and no NaN
+    saturates to scale 448 (0x7E) with code 7 (+6) for +inf; every finite block is the
+    oracle's quantization of the GPU's h; the reported max|h| is NaN, so an amax
+    history rejects it."""
+    K = 256
+    qx, _ = gpu_quantize(synth.activations(31, M, K), nv.SF_MMA)
+    qw, _ = gpu_quantize(synth.weights(31, 0, N, K), nv.SF_MMA)
+    c = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    nv.nvfp4_gemm(qx, qw, c)
+    cmax = float(c.abs().max())
+    qx.gscale.mul_(float(np.float32(3.0e38 / (0.6 * cmax))))  # |c| above ~0.7 max overflows
+    h = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    nv.nvfp4_gemm(qx, qw, None, act=nv.ACT_GELU_TANH, h_out=h)
+    hn = h.cpu().numpy()
+    fin = np.isfinite(hn)
+    assert np.isnan(hn).any() and np.isposinf(hn).any() and fin.mean() > 0.5
+    g_h = np.float32(np.abs(hn[fin]).max() / np.float32(2688.0))
+    q_h = nv.NVFP4Tensor(M, N, nv.SF_MMA)
+    amax = torch.zeros(1, dtype=torch.float32, device="cuda")
+    h2 = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    nv.nvfp4_gemm(qx, qw, None, act=nv.ACT_GELU_TANH, q_out=q_h,
+                  q_gscale_in=torch.tensor([g_h], dtype=torch.float32, device="cuda"),
+                  q_amax_out=amax, h_out=h2)
+    torch.cuda.synchronize()
+    assert device_status() == nv.OK
+    assert np.array_equal(h2.cpu().numpy(), hn, equal_nan=True)
+    assert np.isnan(amax.item())
+    codes, scales, g = canonical(q_h)
+    blocks = hn.reshape(M, N // 16, 16)
+    nan_b = np.isnan(blocks).any(axis=2)
+    inf_b = np.isinf(blocks).any(axis=2) & ~nan_b
+    fin_b = ~(nan_b | inf_b)
+    assert nan_b.any() and inf_b.any() and fin_b.any()
+    assert np.all(scales[nan_b] == 0x7F)
+    assert np.all(scales[inf_b] == 0x7E)
+    nib = np.stack([codes & 0xF, codes >> 4], axis=-1).reshape(M, N)
+    in_inf_b = np.repeat(inf_b, 16, axis=1)
+    assert np.all(nib[np.isposinf(hn) & in_inf_b] == 0x7)
+    assert np.all(nib[np.repeat(nan_b, 16, axis=1)] & 0x7 == 0)  # NaN blocks: signs only
+    hz = np.where(np.repeat(fin_b, 16, axis=1), hn, np.float32(0)).astype(np.float32)
+    ref = oracle.quantize(hz, gscale=float(g_h))
+    assert np.array_equal(scales[fin_b], ref.scales[fin_b])
+    fin_bytes = np.repeat(fin_b, 8, axis=1)
+    assert np.array_equal(codes[fin_bytes], ref.codes[fin_bytes])
+
+
 @pytest.mark.slow
 @pytest.mark.parametrize("K,N", [(3072, 3072), (3072, 9216), (3072, 14336), (14336, 3072)])
 def test_full_size_block_gemms_sampled_rows(cuda_dev, K, N):
