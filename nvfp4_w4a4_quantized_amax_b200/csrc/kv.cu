@@ -70,6 +70,27 @@ struct StatsParams {
   Scratch sc;
 };
 
+__device__ __forceinline__ uint32_t max_s16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("max.s16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t min_s16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.s16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+__device__ __forceinline__ uint32_t min_u16x2(uint32_t a, uint32_t b) {
+  uint32_t r;
+  asm("min.u16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+  return r;
+}
+// bf16 value of an order-preserving int16 key (inverse of the key transform)
+__device__ __forceinline__ float key_to_float(int key) {
+  const uint32_t b = (uint32_t)(key < 0 ? (key ^ 0x7FFF) : key) & 0xFFFFu;
+  return __uint_as_float(b << 16);
+}
+
 __global__ void __launch_bounds__(kStatsThreads) kv_stats_kernel(StatsParams p) {
   pdl_trigger();
   pdl_wait();
@@ -80,17 +101,21 @@ __global__ void __launch_bounds__(kStatsThreads) kv_stats_kernel(StatsParams p) 
   const int64_t t_begin = (int64_t)split * p.tokens_per_split;
   const int64_t t_end = min(p.T, t_begin + p.tokens_per_split);
 
+  // Per lane 8 columns = 4 words of two bf16.  The sums are doubles; max and min of
+  // k are kept as order-preserving int16 keys (key = bits, with the magnitude bits
+  // flipped for negative values) and the smallest nonzero |k| as |k| - 1 mod 2^15
+  // (zero becomes 0x7FFF, above every nonzero magnitude), all two to a register.
   double sum[8];
-  float kmax[8], kmin[8];
-  unsigned amin[8];
+  uint32_t kmx[4], kmn[4], amn[4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    sum[i] = 0.0;
-    kmax[i] = -3.402823466e38f;
-    kmin[i] = 3.402823466e38f;
-    amin[i] = 0xFFFFFFFFu;
+  for (int i = 0; i < 8; ++i) sum[i] = 0.0;
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    kmx[q] = 0x80008000u;
+    kmn[q] = 0x7FFF7FFFu;
+    amn[q] = 0x7FFF7FFFu;
   }
-  unsigned kbad = 0, vmax = 0;
+  unsigned vmax = 0;
   if (active) {
     constexpr int kRowStep = kStatsThreads / 32;
     for (int64_t t0 = t_begin + warp; t0 < t_end; t0 += kRowStep * kStatsUnroll) {
@@ -108,15 +133,14 @@ __global__ void __launch_bounds__(kStatsThreads) kv_stats_kernel(StatsParams p) 
         if (t0 + (int64_t)u * kRowStep >= t_end) break;
         const uint32_t w[4] = {kw[u].x, kw[u].y, kw[u].z, kw[u].w};
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint32_t bits = (i & 1) ? (w[i >> 1] >> 16) : (w[i >> 1] & 0xFFFFu);
-          const float f = __uint_as_float(bits << 16);
-          sum[i] += (double)f;
-          kmax[i] = fmaxf(kmax[i], f);
-          kmin[i] = fminf(kmin[i], f);
-          const unsigned a = (bits & 0x7FFFu) << 16;
-          kbad = max(kbad, a);
-          amin[i] = min(amin[i], a ? a : 0xFFFFFFFFu);
+        for (int q = 0; q < 4; ++q) {
+          const uint32_t x = w[q];
+          sum[2 * q] += (double)__uint_as_float(x << 16);
+          sum[2 * q + 1] += (double)__uint_as_float(x & 0xFFFF0000u);
+          const uint32_t key = x ^ (((x >> 15) & 0x00010001u) * 0x7FFFu);
+          kmx[q] = max_s16x2(kmx[q], key);
+          kmn[q] = min_s16x2(kmn[q], key);
+          amn[q] = min_u16x2(amn[q], ((x & 0x7FFF7FFFu) + 0x7FFF7FFFu) & 0x7FFF7FFFu);
         }
         vmax = __vmaxu2(vmax, vw[u].x & 0x7FFF7FFFu);
         vmax = __vmaxu2(vmax, vw[u].y & 0x7FFF7FFFu);
@@ -124,6 +148,22 @@ __global__ void __launch_bounds__(kStatsThreads) kv_stats_kernel(StatsParams p) 
         vmax = __vmaxu2(vmax, vw[u].w & 0x7FFF7FFFu);
       }
     }
+  }
+  // back to floats and bit patterns per column; a key of +inf or above (+inf, +NaN)
+  // or of -inf or below flags a non-finite k
+  float kmax[8], kmin[8];
+  unsigned amin[8];
+  unsigned kbad = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int sh = 16 * (i & 1);
+    const int hi = (int)(int16_t)(uint16_t)(kmx[i >> 1] >> sh);
+    const int lo = (int)(int16_t)(uint16_t)(kmn[i >> 1] >> sh);
+    const unsigned a16 = (amn[i >> 1] >> sh) & 0xFFFFu;
+    kmax[i] = hi == -32768 ? -3.402823466e38f : key_to_float(hi);
+    kmin[i] = lo == 32767 ? 3.402823466e38f : key_to_float(lo);
+    amin[i] = a16 == 0x7FFFu ? 0xFFFFFFFFu : (a16 + 1u) << 16;
+    if (hi >= 0x7F80 || lo <= (int)(int16_t)0x807F) kbad = 0x7F800000u;
   }
   vmax = max(vmax >> 16, vmax & 0xFFFFu) << 16;
 
@@ -272,6 +312,7 @@ __global__ void __launch_bounds__(kMuThreads) kv_mu_kernel(MuParams p) {
     float mx = -3.402823466e38f, mn = 3.402823466e38f;
     unsigned am = 0xFFFFFFFFu;
     if (c < p.C) {
+#pragma unroll 4
       for (int sp = warp; sp < p.nsplits; sp += kWarps) {
         const int64_t o = (int64_t)sp * p.C + c;
         S += p.sc.sum[o];

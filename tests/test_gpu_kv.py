@@ -88,7 +88,11 @@ def test_wide_range_columns_take_the_exact_path(cuda_dev):
     run_cache(heads=2, head_dim=32, T=64, chunks=2, window=2, seed=4, plant=plant)
 
 
-def test_nonfinite_chunk_leaves_slot_unchanged(cuda_dev):
+@pytest.mark.parametrize("where,bits", [("v", 0x7F80), ("v", 0xFF80), ("v", 0x7FC0),
+                                        ("k", 0x7F80), ("k", 0xFF80), ("k", 0x7FC0), ("k", 0xFFC1)])
+def test_nonfinite_chunk_leaves_slot_unchanged(cuda_dev, where, bits):
+    """+-inf and +-NaN in K or V: NONFINITE in the device status, the slot keeps its
+    previous contents."""
     heads, dh, T = 2, 32, 64
     off = synth.kv_offsets(1, heads, dh)
     cache = nv.KVCache(heads, dh, T, 2)
@@ -97,10 +101,30 @@ def test_nonfinite_chunk_leaves_slot_unchanged(cuda_dev):
     ref = oracle.kv_append(k, v)
     device_status(clear=True)
     k2, v2 = synth.kv_chunk(1, 1, T, heads, dh, off)
-    v2[7, 1, 3] = 0x7F80  # +inf
+    (v2 if where == "v" else k2)[7, 1, 3] = bits
+    with pytest.raises(FloatingPointError):  # the oracle rejects the chunk too
+        oracle.kv_append(k2, v2)
     nv.kv_quant_append(cache, dev_bf16(k2), dev_bf16(v2), 0)
     assert device_status(clear=True) == nv.ERR_NONFINITE
     check_slot(cache, 0, ref)
+
+
+def test_signed_zero_and_one_signed_columns(cuda_dev):
+    """Columns of -0 only, of +0 and -0, of negative values only, of positive values
+    only, and of subnormals only: max, min, mean and the smallest nonzero magnitude
+    of every column as the oracle has them."""
+    def plant(c, k, v):
+        flat = k.reshape(k.shape[0], -1)
+        flat[:, 50] = 0x8000                 # -0 everywhere
+        flat[:, 51] = 0x8000
+        flat[::2, 51] = 0x0000               # +0 and -0
+        flat[:, 52] = 0xBF80                 # -1 ...
+        flat[::3, 52] = 0xC040               # ... and -3
+        flat[:, 53] = 0x3F80                 # +1 ...
+        flat[1::4, 53] = 0x4100              # ... and +8
+        flat[:, 54] = 0x0003                 # subnormals ...
+        flat[::5, 54] = 0x8005               # ... of both signs
+    run_cache(heads=2, head_dim=32, T=64, chunks=2, window=2, seed=6, plant=plant)
 
 
 @pytest.mark.slow
