@@ -128,16 +128,6 @@ static __device__ __noinline__ uint32_t e2m1_index_exact_f64(float ax, float D) 
   return i;
 }
 
-// Hardware RNE of two floats onto E2M1 (saturating at 6): `lo` in bits 0..3.
-__device__ __forceinline__ uint32_t e2m1x2_rn(float lo, float hi) {
-  uint32_t r;
-  asm("{\n\t.reg .b8 t;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
-      "cvt.u32.u8 %0, t;\n\t}"
-      : "=r"(r)
-      : "f"(hi), "f"(lo));
-  return r;
-}
 
 // Block encoder: D = RN(s * g) and rD ~ 1 / D (hardware reciprocal, <= 1 ulp) are
 // computed once per block, and from rD two brackets rDlo < 1 / D < rDhi (rD scaled
@@ -196,10 +186,18 @@ __device__ __forceinline__ uint32_t f32_signs8(const float (&v)[8]) {
   return r;
 }
 
+// 8 values -> 8 codes, element k in bits 4k..4k+3: four paired conversions whose
+// bytes are packed by one vector move.
 __device__ __forceinline__ uint32_t pack_e2m1x8(const float (&q)[8]) {
-  uint32_t word = 0;
-#pragma unroll
-  for (int k = 0; k < 8; k += 2) word |= e2m1x2_rn(q[k], q[k + 1]) << (4 * k);
+  uint32_t word;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(word)
+      : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
   return word;
 }
 
