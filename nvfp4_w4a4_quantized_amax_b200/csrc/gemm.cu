@@ -283,12 +283,19 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
 // with the hardware exp2 and reciprocal approximations (relative error ~2^-22 over
 // the binary32 range against the 2^-16 (|c| + |h|) the GEMM promises for h; large
 // |c| gives h = c or -0, infinities as the formula).
-__device__ __forceinline__ float gelu_tanh(float c) {
-  const float x = c * fmaf(c * c, -0.1029432396f, -2.3022081983f);
-  float e, r;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(x));
-  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.0f + e));
-  return c * r;
+// Two values at a time: the FP32 steps as two-lane operations (same roundings as the
+// scalar form), exp2 and reciprocal per value.
+__device__ __forceinline__ void gelu_tanh2(float& c0, float& c1) {
+  float t0, t1, u0, u1, x0, x1, e0, e1, d0, d1, r0, r1;
+  mul2(t0, t1, c0, c1, c0, c1);
+  fma2(u0, u1, t0, t1, -0.1029432396f, -0.1029432396f, -2.3022081983f, -2.3022081983f);
+  mul2(x0, x1, c0, c1, u0, u1);
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e0) : "f"(x0));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e1) : "f"(x1));
+  add2(d0, d1, 1.0f, 1.0f, e0, e1);
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(d0));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r1) : "f"(d1));
+  mul2(c0, c1, c0, c1, r0, r1);
 }
 
 // ----------------------------------------------------------------- the kernel
@@ -508,10 +515,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (col0 >= p.N) continue;  // warp-uniform
         float v[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]) * gab;
+        for (int i = 0; i < 32; i += 2)
+          mul2(v[i], v[i + 1], __uint_as_float(r[i]), __uint_as_float(r[i + 1]), gab, gab);
         if (p.act == 1) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
+          for (int i = 0; i < 32; i += 2) gelu_tanh2(v[i], v[i + 1]);
         }
         if (p.c) {
           // Stage this warp's 32 rows x 32 columns in shared memory (swizzled like the
@@ -1039,10 +1047,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         if (col0 >= p.N) break;  // warp-uniform
         float* v = reinterpret_cast<float*>(r[h]);
 #pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[h][i]) * gab;
+        for (int i = 0; i < 32; i += 2)
+          mul2(v[i], v[i + 1], __uint_as_float(r[h][i]), __uint_as_float(r[h][i + 1]), gab, gab);
         if (kFused && p.act == 1) {
 #pragma unroll
-          for (int i = 0; i < 32; ++i) v[i] = gelu_tanh(v[i]);
+          for (int i = 0; i < 32; i += 2) gelu_tanh2(v[i], v[i + 1]);
         }
         if (has_c) {
           if (p.c_bf16) {

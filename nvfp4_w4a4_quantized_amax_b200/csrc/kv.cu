@@ -430,8 +430,10 @@ __device__ __forceinline__ void encode_block16(const float (&v)[16], float g, fl
   const uint32_t s = block_scale_fast(amax_b, d6, r6);
   const BlockEncoder enc(e4m3_to_float(s) * g);
   uint2 out;
-  out.x = enc.encode8s(v0);
-  out.y = enc.encode8s(v1);
+  // scalar bracket products here: the paired form costs this kernel a resident CTA
+  // per SM (66 registers), which measured slower
+  out.x = enc.encode8s<false>(v0);
+  out.y = enc.encode8s<false>(v1);
   stg_v2(codes, out);
   *scale = (uint8_t)s;
 }
