@@ -629,18 +629,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ============================================================ 2-CTA pair kernel
-// One cluster of 2 CTAs computes a 256 x 128 tile with tcgen05.mma.cta_group::2:
-// CTA r of the pair holds rows [128 r, 128 r + 128) of the A tile and rows
-// [64 r, 64 r + 64) of the W tile in its shared memory, and rows 128 r .. of the
-// accumulator in its tensor memory.  The even CTA issues every MMA; operands are
-// read from both CTAs' shared memory by the hardware.  Each CTA loads only its
-// own halves (no TMA multicast): 24 KB of codes per 256 K values per CTA for a
-// 128 x 128 share of the output, against 32 KB for a 128 x 128 tile of one CTA.
+// One cluster of 2 CTAs computes a 256 x kBN tile (kBN = 256) with
+// tcgen05.mma.cta_group::2 (M = 256, N = kBN, K = 64 per instruction): CTA r of the
+// pair holds rows [128 r, 128 r + 128) of the A tile and rows [r kBN/2, (r + 1) kBN/2)
+// of the W tile in its shared memory, and rows 128 r .. of the accumulator in its
+// tensor memory.  The even CTA issues every MMA; operands are read from both CTAs'
+// shared memory by the hardware.  Each CTA loads only its own halves (no TMA
+// multicast): 32 KB of codes per 256 K values per CTA for a 128 x 256 share of the
+// output, against 48 KB for a 128 x 256 tile of one CTA.
 //
-// Tensor memory per CTA (512 columns): accumulators 2 x 128, then one scale slot
-// per pipeline stage of 4 MMAs x 8 columns: [A scales 0..3 | W scales 4..7]; the
-// W scales of all 128 rows are present in both CTAs (the hardware reads them in
-// the SM that holds the accumulator rows).
+// Tensor memory per CTA (512 columns): kAccStages accumulators of kBN columns (one
+// at kBN = 256), then one scale slot per pipeline stage of 4 MMAs x (4 + 4 kWTiles)
+// columns: per MMA [A scales | W scales of each 128-row W tile]; the W scales of all
+// kBN rows are present in both CTAs (the hardware reads them in the SM that holds
+// the accumulator rows).
 namespace pair {
 
 constexpr int kBM = 256;            // rows per pair tile (128 per CTA)
