@@ -10,7 +10,9 @@
 //   c[m, n] = RN(acc[m, n] * RN(gA * gW)),   C = act(c)  (act: none or GELU-tanh)
 //   acc     = sum_k (e2m1(A[m,k]) sA[m,k/16]) (e2m1(W[n,k]) sW[n,k/16])  (FP32, tensor core)
 //
-// Structure: one persistent CTA per SM, 6 warps.
+// Two kernels.  gemm_kernel (below): one persistent CTA per SM, 128 x 128 tiles,
+// 14 warps.  gemm_pair_kernel (further down): CTA pairs, 256 x 256 tiles, 24 warps.
+// Structure of gemm_kernel:
 //   warp 0      TMA producer: A and W code tiles (128 B swizzle, 128 rows x 256
 //               values per stage) and the stage's scale atoms (bulk copies).
 //   warp 1      MMA issuer: tcgen05.mma.kind::mxf4nvf4.block_scale (UE4M3,
