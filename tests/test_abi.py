@@ -137,3 +137,48 @@ def test_host_argument_checks_return_before_any_device_work():
     assert Hp(None, 4, p, p, None) == nv.ERR_INVALID_ARG
     assert Hp(p, 0, p, p, None) == nv.ERR_SHAPE
     assert Hp(p, 1025, p, p, None) == nv.ERR_SHAPE
+
+
+def test_dequantize_and_gemm_epilogue_host_checks():
+    """The argument rules of nvfp4_dequantize and of the GEMM epilogue, each checked on
+    the host (no device is touched: every call returns before the device lookup)."""
+    lib = nv.library()
+    p = ctypes.c_void_p(4096)
+    t = _fake_tensor(16, 64)
+    D = lib.nvfp4_dequantize
+    assert D(ctypes.byref(t), None, nv.BF16, 64, None) == nv.ERR_INVALID_ARG      # no output
+    assert D(ctypes.byref(t), p, 7, 64, None) == nv.ERR_INVALID_ARG                # output dtype
+    assert D(ctypes.byref(t), p, nv.BF16, 48, None) == nv.ERR_SHAPE                # ldy < cols
+    assert D(ctypes.byref(t), ctypes.c_void_p(4100), nv.FP32, 64, None) == nv.ERR_ALIGNMENT
+    assert D(ctypes.byref(t), p, nv.BF16, 68, None) == nv.ERR_ALIGNMENT           # row pitch 136 B
+
+    G = lib.nvfp4_gemm
+    a = _fake_tensor(64, 64)
+    w = _fake_tensor(128, 64)
+    w40 = _fake_tensor(40, 64)
+    ok = lambda ep, c=p, ct=nv.FP32, ldc=128, W=w: G(ctypes.byref(a), ctypes.byref(W), c, ct, ldc,  # noqa: E731
+                                                     None if ep is None else ctypes.byref(ep), None)
+    assert ok(None, W=w40, ldc=40) == nv.ERR_SHAPE                  # N % 16 != 0
+    assert ok(None, ldc=120) == nv.ERR_SHAPE                         # ldc < N
+    assert ok(None, c=ctypes.c_void_p(4104)) == nv.ERR_ALIGNMENT     # C not 16-byte aligned
+    assert ok(None, ct=9) == nv.ERR_INVALID_ARG                      # C dtype
+    assert ok(None, c=None) == nv.ERR_INVALID_ARG                    # no output at all
+    ep = nv.nvfp4_epilogue(5, 0, None, None, None, None)
+    assert ok(ep) == nv.ERR_INVALID_ARG                              # unknown activation
+    ep = nv.nvfp4_epilogue(nv.ACT_GELU_TANH, 1, None, None, None, None)
+    assert ok(ep) == nv.ERR_INVALID_ARG                              # reserved field set
+    q = _fake_tensor(64, 128)
+    ep = nv.nvfp4_epilogue(nv.ACT_GELU_TANH, 0, ctypes.pointer(q), None, None, None)
+    assert ok(ep, c=None) == nv.ERR_INVALID_ARG                      # q_out without its scale
+    qr = _fake_tensor(64, 128, nv.SF_ROWMAJOR)
+    ep = nv.nvfp4_epilogue(nv.ACT_GELU_TANH, 0, ctypes.pointer(qr), p, None, None)
+    assert ok(ep, c=None) == nv.ERR_INVALID_ARG                      # q_out must use the MMA layout
+    q_small = _fake_tensor(32, 128)
+    ep = nv.nvfp4_epilogue(nv.ACT_GELU_TANH, 0, ctypes.pointer(q_small), p, None, None)
+    assert ok(ep, c=None) == nv.ERR_SHAPE                            # q_out is not [M, N]
+    w48 = _fake_tensor(48, 64)
+    q48 = _fake_tensor(64, 48)
+    ep = nv.nvfp4_epilogue(nv.ACT_GELU_TANH, 0, ctypes.pointer(q48), p, None, None)
+    assert ok(ep, c=None, W=w48, ldc=48) == nv.ERR_SHAPE             # requantization needs N % 64 == 0
+    ep = nv.nvfp4_epilogue(nv.ACT_GELU_TANH, 0, None, None, None, ctypes.c_void_p(4098))
+    assert ok(ep, c=None) == nv.ERR_ALIGNMENT                        # h_out not 16-byte aligned
