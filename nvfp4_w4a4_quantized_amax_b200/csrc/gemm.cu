@@ -1174,13 +1174,16 @@ typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 
 EncodeTiledFn get_encode_fn() {
-  static EncodeTiledFn fn = nullptr;
+  static std::atomic<EncodeTiledFn> cached{nullptr};
+  EncodeTiledFn fn = cached.load(std::memory_order_relaxed);
   if (!fn) {
     void* ptr = nullptr;
     cudaDriverEntryPointQueryResult q;
     if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
+        q == cudaDriverEntryPointSuccess) {
       fn = reinterpret_cast<EncodeTiledFn>(ptr);
+      cached.store(fn, std::memory_order_relaxed);
+    }
   }
   return fn;
 }
@@ -1224,15 +1227,15 @@ bool make_out_map(CUtensorMap* m, void* base, int64_t rows, int64_t cols, int64_
 
 // Opt a kernel into its dynamic shared memory once per device.
 template <typename Kernel>
-cudaError_t set_smem_once(Kernel k, int bytes, bool (&done)[64]) {
+cudaError_t set_smem_once(Kernel k, int bytes, std::atomic<bool> (&done)[64]) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!done[dev]) {
+  if (!done[dev].load(std::memory_order_relaxed)) {  // setting it twice is harmless
     e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
-    done[dev] = true;
+    done[dev].store(true, std::memory_order_relaxed);
   }
   return cudaSuccess;
 }
@@ -1287,17 +1290,17 @@ cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s) {
     cudaError_t e = launch_zero_words(g.q_amax_out, 1, s);
     if (e != cudaSuccess) return e;
   }
-  static bool done[64];
+  static std::atomic<bool> done[64];
   cudaError_t e = set_smem_once(pair::gemm_pair_kernel<kFused>, pair::kSmemBytes, done);
   if (e != cudaSuccess) return e;
   // Pairs must fit inside one GPC, so fewer than SMs / 2 of them may be resident
   // at once; a persistent grid larger than that would run a second wave.
-  static int resident[64];
+  static std::atomic<int> resident[64];
   int dev = 0;
   e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (resident[dev] == 0) {
+  if (resident[dev].load(std::memory_order_relaxed) == 0) {
     // The kernel's register split (setmaxnreg) balances only for this launch count:
     // with fewer registers at launch its epilogue warps would wait for registers
     // that are never released.
@@ -1321,9 +1324,9 @@ cudaError_t launch_gemm_pair(const GemmArgs& g, cudaStream_t s) {
     e = cudaOccupancyMaxActiveClusters(&n, pair::gemm_pair_kernel<kFused>, &cfg);
     if (e != cudaSuccess) return e;
     if (n <= 0) return cudaErrorInvalidConfiguration;
-    resident[dev] = n;
+    resident[dev].store(n, std::memory_order_relaxed);
   }
-  const int64_t max_pairs = resident[dev];
+  const int64_t max_pairs = resident[dev].load(std::memory_order_relaxed);
   const int64_t pairs = p.num_tiles < max_pairs ? p.num_tiles : max_pairs;
   launch_pdl(pair::gemm_pair_kernel<kFused>, (unsigned)(2 * pairs), pair::kThreads, pair::kSmemBytes, s, ma, mw, mc, p);
   return cudaGetLastError();
@@ -1379,7 +1382,7 @@ cudaError_t launch_gemm(const GemmArgs& g, cudaStream_t s) {
     cudaError_t e = launch_zero_words(g.q_amax_out, 1, s);
     if (e != cudaSuccess) return e;
   }
-  static bool done[64];
+  static std::atomic<bool> done[64];
   cudaError_t e = set_smem_once(gemm_kernel, kSmemBytes, done);
   if (e != cudaSuccess) return e;
   const int sms = sm_count_gemm();

@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <atomic>
+
 namespace nvfp4 {
 
 // Launch with programmatic stream serialization (the kernel calls pdl_trigger and
@@ -32,16 +34,19 @@ cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t s
 // exactly one full wave.
 template <auto K>
 int resident_ctas(int threads) {
-  static int cache[64];
+  // per device; host threads may race on the first call, all writing the same value
+  static std::atomic<int> cache[64];
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
-  if (cache[dev] == 0) {
+  int n = cache[dev].load(std::memory_order_relaxed);
+  if (n == 0) {
     int per_sm = 0, sms = 148;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, K, threads, 0) != cudaSuccess) per_sm = 1;
     cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    cache[dev] = (per_sm > 0 ? per_sm : 1) * sms;
+    n = (per_sm > 0 ? per_sm : 1) * sms;
+    cache[dev].store(n, std::memory_order_relaxed);
   }
-  return cache[dev];
+  return n;
 }
 
 // One wave of K, or fewer CTAs when `work` items (one per thread) need fewer.

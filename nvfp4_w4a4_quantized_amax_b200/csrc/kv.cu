@@ -579,19 +579,20 @@ int sm_count() {
 cudaError_t launch_append_kernels(const KVLayout& L, const void* k, const void* v, int64_t T, int32_t slot,
                                   const Scratch& sc, unsigned* status, cudaStream_t s) {
   const int64_t C = (int64_t)L.heads * L.head_dim;
-  static int resident[64];
+  static std::atomic<int> resident[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (resident[dev] == 0) {
+  if (resident[dev].load(std::memory_order_relaxed) == 0) {
     int per_sm = 0;
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kv_stats_kernel, kStatsThreads, 0);
     if (e != cudaSuccess) return e;
-    resident[dev] = max(1, per_sm) * sm_count();
+    resident[dev].store(max(1, per_sm) * sm_count(), std::memory_order_relaxed);
   }
   const int64_t colblocks = (C + kStatsCols - 1) / kStatsCols;
-  const int nsplits = (int)max((int64_t)1, min((int64_t)kSplits, resident[dev] / colblocks));
+  const int64_t resident_now = resident[dev].load(std::memory_order_relaxed);
+  const int nsplits = (int)max((int64_t)1, min((int64_t)kSplits, resident_now / colblocks));
 
   StatsParams sp;
   sp.k = (const uint8_t*)k;
