@@ -122,6 +122,25 @@ nvfp4_status nvfp4_quantize(const void* x, int32_t xt, int64_t rows, int64_t col
                             const float* gscale_in, const nvfp4_tensor* out, float* amax_out,
                             nvfp4_stream_t stream);
 
+/* nvfp4_amax — max |x| over a whole tensor (the first step of quantization, alone).
+ * [TW] §一: the tensor shares one FP32 scale; the library takes it as
+ * g = RN(amax / 2688).  On its own this serves a tensor whose rows are split
+ * across GPUs: each GPU takes the amax of its rows, the GPUs combine them with an
+ * all-reduce(MAX) -- exact and independent of order; done on the binary32 bit
+ * patterns as signed 32-bit integers it also carries a NaN through -- and each
+ * quantizes its rows with nvfp4_quantize(gscale_in = RN(amax / 2688)), for which
+ * nvfp4_amax_history_push with a one-entry history computes g on the device.  The
+ * codes and scales of every row are then bit-identical to quantizing the whole
+ * tensor on one GPU.
+ *   x        : device, row-major [rows, cols] of xt (NVFP4_BF16 or NVFP4_FP32), ldx
+ *              elements (>= cols), cols % 16 == 0; base and row pitch 16-byte
+ *              aligned; may be NULL when rows == 0 (amax = 0).
+ *   amax_out : device FP32 [1]: max|x| (its bits are those of the largest |x|, so
+ *              an Inf gives +inf and a NaN a NaN).
+ * Errors: INVALID_ARG (NULL, bad dtype), SHAPE, ALIGNMENT. */
+nvfp4_status nvfp4_amax(const void* x, int32_t xt, int64_t rows, int64_t cols, int64_t ldx, float* amax_out,
+                        nvfp4_stream_t stream);
+
 /* nvfp4_dequantize — y = RN(RN(e2m1 * s) * g), stored as FP32 or as bf16 (RNE).
  * [TW] §一 (format).  y: device row-major [rows, cols], leading dimension ldy
  * elements, 16-byte aligned base and row pitch.  Either scale layout. */
@@ -209,7 +228,12 @@ nvfp4_status nvfp4_kv_cache_bytes(int32_t heads, int32_t head_dim, int64_t chunk
 
 /* Lays out a cache in caller-owned device memory `dev_mem` (256-byte aligned,
  * `bytes` >= nvfp4_kv_cache_bytes(...)) and fills the host struct `cache`.
- * No device work is enqueued; slots hold garbage until appended. */
+ * No device work is enqueued; slots hold garbage until appended.
+ * A caller that appends only with kv_quant_append_noalloc may give a shorter
+ * allocation that ends at cache->off_scratch (the append scratch is then absent:
+ * kv_quant_append returns NVFP4_ERR_INVALID_ARG on such a cache, while
+ * kv_quant_append_noalloc and the window calls accept it).  Below off_scratch:
+ * NVFP4_ERR_SHAPE. */
 nvfp4_status nvfp4_kv_cache_init(void* dev_mem, size_t bytes, int32_t heads, int32_t head_dim,
                                  int64_t chunk_tokens, int32_t max_chunks, nvfp4_kv_cache* cache);
 
@@ -232,7 +256,9 @@ nvfp4_status kv_quant_append(const nvfp4_kv_cache* cache, const void* k, const v
  * entry point allocates nothing and needs no scratch from the caller: the
  * per-chunk column statistics live in one static device array of the library
  * (about 5 MiB, present on every device that loads the library until the
- * process exits), not in the cache's scratch region, which it never touches.
+ * process exits), not in the cache's scratch region, which it never touches —
+ * the cache may be laid out in an allocation that stops at off_scratch (see
+ * nvfp4_kv_cache_init).
  * Inputs and outputs are exactly those of kv_quant_append and the slot it writes
  * is bit-identical.
  *   Limit: heads * head_dim <= NVFP4_NOALLOC_MAX_COLUMNS, else NVFP4_ERR_SHAPE.
@@ -242,7 +268,11 @@ nvfp4_status kv_quant_append(const nvfp4_kv_cache* cache, const void* k, const v
  *   Sharing: every call on a device uses the same array and it keeps the last
  *   call's contents; the call clears what must start at zero itself.  Calls whose
  *   work overlaps on the GPU (other streams, other threads) race on the array:
- *   issue them on one stream or serialize them. */
+ *   issue them on one stream or serialize them.
+ *   Device reset: the library keeps the array's device address (and that of the
+ *   device status word) per device for the life of the process; after
+ *   cudaDeviceReset on a device those cached addresses are stale, so do not call
+ *   into the library on that device again in the same process. */
 #define NVFP4_NOALLOC_MAX_COLUMNS 4096
 nvfp4_status kv_quant_append_noalloc(const nvfp4_kv_cache* cache, const void* k, const void* v,
                                      int64_t tokens, int32_t slot, nvfp4_stream_t stream);

@@ -150,6 +150,28 @@ nvfp4_status nvfp4_quantize(const void* x, int32_t xt, int64_t rows, int64_t col
   return cuda_status(nvfp4::launch_quantize(a, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_amax(const void* x, int32_t xt, int64_t rows, int64_t cols, int64_t ldx, float* amax_out,
+                        nvfp4_stream_t stream) {
+  if ((!x && rows > 0) || !amax_out || !valid_dtype(xt)) return NVFP4_ERR_INVALID_ARG;
+  if (rows < 0 || cols <= 0 || cols % 16 != 0 || (rows > 0 && ldx < cols)) return NVFP4_ERR_SHAPE;
+  const int64_t esz = xt == NVFP4_BF16 ? 2 : 4;
+  if (rows > 0 && (!aligned16(x) || (ldx * esz) % 16 != 0)) return NVFP4_ERR_ALIGNMENT;
+  if (reinterpret_cast<uintptr_t>(amax_out) & 3u) return NVFP4_ERR_ALIGNMENT;
+  if (rows * cols * esz / 16 >= kMaxBlocks) return NVFP4_ERR_SHAPE;
+  unsigned* status = nullptr;
+  nvfp4_status st = current_device(&status);
+  if (st != NVFP4_OK) return st;
+  nvfp4::QuantizeArgs a = {};
+  a.x = x;
+  a.x_bf16 = xt == NVFP4_BF16;
+  a.rows = rows;
+  a.cols = cols;
+  a.ldx = ldx;
+  a.amax_out = amax_out;
+  a.status = status;
+  return cuda_status(nvfp4::launch_amax(a, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_dequantize(const nvfp4_tensor* in, void* y, int32_t yt, int64_t ldy,
                               nvfp4_stream_t stream) {
   nvfp4_status st = check_tensor(in);
@@ -273,7 +295,9 @@ nvfp4_status nvfp4_kv_cache_init(void* dev_mem, size_t bytes, int32_t heads, int
   size_t need = 0;
   nvfp4_status st = kv_geometry(heads, head_dim, chunk_tokens, max_chunks, &L, &need);
   if (st != NVFP4_OK) return st;
-  if (bytes < need) return NVFP4_ERR_SHAPE;
+  // an allocation that ends before the append scratch serves kv_quant_append_noalloc
+  // and the window calls; kv_quant_append then returns INVALID_ARG
+  if (bytes < (size_t)L.off_scratch) return NVFP4_ERR_SHAPE;
   cache->base = static_cast<uint8_t*>(dev_mem);
   cache->bytes = bytes;
   cache->heads = heads;
@@ -294,12 +318,15 @@ nvfp4_status nvfp4_kv_cache_init(void* dev_mem, size_t bytes, int32_t heads, int
   return NVFP4_OK;
 }
 
-// Re-derives the layout from the geometry and checks it against the handle.
-static nvfp4_status check_cache(const nvfp4_kv_cache* c, nvfp4::KVLayout* L) {
+// Re-derives the layout from the geometry and checks it against the handle.  A
+// caller that never uses the cache's append scratch (kv_quant_append_noalloc) may
+// hand over an allocation that ends where the scratch region would begin.
+static nvfp4_status check_cache(const nvfp4_kv_cache* c, nvfp4::KVLayout* L, bool needs_scratch = true) {
   if (!c || !c->base) return NVFP4_ERR_INVALID_ARG;
   size_t need = 0;
   nvfp4_status st = kv_geometry(c->heads, c->head_dim, c->chunk_tokens, c->max_chunks, L, &need);
   if (st != NVFP4_OK) return st;
+  if (!needs_scratch) need = (size_t)L->off_scratch;
   if (c->bytes < need || L->off_scratch != c->off_scratch || L->off_mu != c->off_mu ||
       L->off_tokens != c->off_tokens)
     return NVFP4_ERR_INVALID_ARG;
@@ -325,7 +352,7 @@ nvfp4_status kv_quant_append(const nvfp4_kv_cache* cache, const void* k, const v
 nvfp4_status kv_quant_append_noalloc(const nvfp4_kv_cache* cache, const void* k, const void* v,
                                      int64_t tokens, int32_t slot, nvfp4_stream_t stream) {
   nvfp4::KVLayout L;
-  nvfp4_status st = check_cache(cache, &L);
+  nvfp4_status st = check_cache(cache, &L, /*needs_scratch=*/false);
   if (st != NVFP4_OK) return st;
   if (!k || !v) return NVFP4_ERR_INVALID_ARG;
   if (!aligned16(k) || !aligned16(v)) return NVFP4_ERR_ALIGNMENT;
@@ -342,7 +369,7 @@ nvfp4_status kv_dequant_window_tokens(const nvfp4_kv_cache* cache, const int32_t
                                       const int32_t* tokens_host, int32_t n_slots, void* k_out,
                                       void* v_out, nvfp4_stream_t stream) {
   nvfp4::KVLayout L;
-  nvfp4_status st = check_cache(cache, &L);
+  nvfp4_status st = check_cache(cache, &L, /*needs_scratch=*/false);
   if (st != NVFP4_OK) return st;
   if (!slots_host || !tokens_host || !k_out || !v_out) return NVFP4_ERR_INVALID_ARG;
   if (n_slots < 1 || n_slots > nvfp4::kMaxWindowSlots) return NVFP4_ERR_INVALID_ARG;

@@ -182,3 +182,21 @@ def test_dequantize_and_gemm_epilogue_host_checks():
     assert ok(ep, c=None, W=w48, ldc=48) == nv.ERR_SHAPE             # requantization needs N % 64 == 0
     ep = nv.nvfp4_epilogue(nv.ACT_GELU_TANH, 0, None, None, None, ctypes.c_void_p(4098))
     assert ok(ep, c=None) == nv.ERR_ALIGNMENT                        # h_out not 16-byte aligned
+
+
+def test_noalloc_cache_may_end_at_the_scratch_region():
+    """A cache laid out without the append scratch: accepted by the no-alloc append
+    (which then fails later, here on a misaligned K, i.e. after the cache check) and
+    refused by kv_quant_append, which needs that scratch.  Host checks only."""
+    lib = nv.library()
+    h = nv.nvfp4_kv_cache()
+    full = ctypes.c_size_t()
+    assert lib.nvfp4_kv_cache_bytes(2, 16, 64, 2, ctypes.byref(full)) == nv.OK
+    assert lib.nvfp4_kv_cache_init(ctypes.c_void_p(4096), full.value, 2, 16, 64, 2, ctypes.byref(h)) == nv.OK
+    short = h.off_scratch
+    assert 0 < short < full.value
+    assert lib.nvfp4_kv_cache_init(ctypes.c_void_p(4096), short - 1, 2, 16, 64, 2, ctypes.byref(h)) == nv.ERR_SHAPE
+    assert lib.nvfp4_kv_cache_init(ctypes.c_void_p(4096), short, 2, 16, 64, 2, ctypes.byref(h)) == nv.OK
+    k = ctypes.c_void_p(4097)
+    assert lib.kv_quant_append(ctypes.byref(h), k, k, 64, 0, None) == nv.ERR_INVALID_ARG
+    assert lib.kv_quant_append_noalloc(ctypes.byref(h), k, k, 64, 0, None) == nv.ERR_ALIGNMENT
