@@ -64,7 +64,7 @@ class nvfp4_kv_cache(ctypes.Structure):
                 ("slot_scales_bytes", ctypes.c_int64)]
 
 
-EXPORTS = ["nvfp4_version", "nvfp4_status_string", "nvfp4_scales_bytes", "nvfp4_quantize",
+EXPORTS = ["nvfp4_version", "nvfp4_status_string", "nvfp4_scales_bytes", "nvfp4_quantize", "nvfp4_amax",
            "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_cache_bytes", "nvfp4_kv_cache_init",
            "kv_quant_append", "kv_quant_append_noalloc", "kv_dequant_window", "kv_dequant_window_tokens",
            "nvfp4_lora_merge", "nvfp4_amax_history_push", "nvfp4_last_cuda_error_string",
@@ -95,6 +95,8 @@ def library():
             lib.nvfp4_scales_bytes.argtypes = [i64, i64, i32, ctypes.POINTER(ctypes.c_size_t)]
             lib.nvfp4_quantize.restype = i32
             lib.nvfp4_quantize.argtypes = [vp, i32, i64, i64, i64, vp, T, vp, vp]
+            lib.nvfp4_amax.restype = i32
+            lib.nvfp4_amax.argtypes = [vp, i32, i64, i64, i64, vp, vp]
             lib.nvfp4_dequantize.restype = i32
             lib.nvfp4_dequantize.argtypes = [T, vp, i32, i64, vp]
             lib.nvfp4_gemm.restype = i32
@@ -191,6 +193,13 @@ def nvfp4_quantize(x, out: NVFP4Tensor, gscale_in=None, amax_out=None, stream=No
     _check(library().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(gscale_in),
                                     ctypes.byref(out.c), _ptr(amax_out), _stream(stream)),
            "nvfp4_quantize")
+
+
+def nvfp4_amax(x, amax_out, stream=None):
+    """max|x| of x [rows, cols] (bf16 or fp32, CUDA) into amax_out (fp32 [1], CUDA)."""
+    rows, cols = x.shape
+    _check(library().nvfp4_amax(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(amax_out),
+                                _stream(stream)), "nvfp4_amax")
 
 
 def nvfp4_dequantize(t: NVFP4Tensor, y, stream=None):

@@ -72,6 +72,8 @@ struct QuantizeArgs {
   unsigned* status;
 };
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s);
+// The amax pass of quantize alone (uses x, x_bf16, rows, cols, ldx, amax_out).
+cudaError_t launch_amax(const QuantizeArgs& a, cudaStream_t s);
 
 struct DequantizeArgs {
   const uint8_t* codes;

@@ -260,6 +260,27 @@ __global__ void __launch_bounds__(kHistThreads) amax_history_kernel(float* histo
 
 }  // namespace
 
+// The amax pass alone: max|x| as binary32 bits into amax_bits (zeroed first).
+static cudaError_t launch_amax_pass(const void* x, bool x_bf16, int64_t rows, int64_t cols, int64_t ldx,
+                                    unsigned* amax_bits, cudaStream_t s) {
+  const int64_t esz = x_bf16 ? 2 : 4;
+  const int64_t cpr = cols * esz / 16;
+  const int64_t n = rows * cpr;
+  if (x_bf16)
+    launch_pdl(amax_kernel<true>, wave_grid<amax_kernel<true>>(kThreads, n), kThreads, 0, s, (const uint8_t*)x,
+               ldx * esz, n, FastDiv((uint32_t)cpr), amax_bits);
+  else
+    launch_pdl(amax_kernel<false>, wave_grid<amax_kernel<false>>(kThreads, n), kThreads, 0, s, (const uint8_t*)x,
+               ldx * esz, n, FastDiv((uint32_t)cpr), amax_bits);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_amax(const QuantizeArgs& a, cudaStream_t s) {
+  cudaError_t e = launch_zero_words(a.amax_out, 1, s);
+  if (e != cudaSuccess || a.rows == 0) return e;
+  return launch_amax_pass(a.x, a.x_bf16, a.rows, a.cols, a.ldx, reinterpret_cast<unsigned*>(a.amax_out), s);
+}
+
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
   const int64_t esz = a.x_bf16 ? 2 : 4;
   const int64_t nb = a.cols / 16;
@@ -275,15 +296,7 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
     return cudaMemcpyAsync(a.gscale_out, a.gscale_in, sizeof(float), cudaMemcpyDeviceToDevice, s);
   }
   if (!a.gscale_in) {
-    const int64_t cpr = a.cols * esz / 16;
-    const int64_t n = a.rows * cpr;
-    if (a.x_bf16)
-      launch_pdl(amax_kernel<true>, wave_grid<amax_kernel<true>>(kThreads, n), kThreads, 0, s, (const uint8_t*)a.x, a.ldx * esz, n,
-                                                         FastDiv((uint32_t)cpr), amax_bits);
-    else
-      launch_pdl(amax_kernel<false>, wave_grid<amax_kernel<false>>(kThreads, n), kThreads, 0, s, (const uint8_t*)a.x, a.ldx * esz, n,
-                                                          FastDiv((uint32_t)cpr), amax_bits);
-    cudaError_t e = cudaGetLastError();
+    cudaError_t e = launch_amax_pass(a.x, a.x_bf16, a.rows, a.cols, a.ldx, amax_bits, s);
     if (e != cudaSuccess) return e;
   }
   EncodeParams p;
