@@ -163,14 +163,40 @@ def fused_case(M, N, K, seed):
     return c.cpu().numpy(), h2.cpu().numpy(), q_h, float(g_h), float(amax2.item()), h.cpu().numpy()
 
 
+# GELU_tanh(c) = c / (1 + 2^X(c)) with X(c) = c (A c^2 + B), B = -2 sqrt(2/pi) log2(e),
+# A = 0.044715 B (float64 here; the epilogue evaluates the same form in binary32).
+_GELU_B = -2.0 * np.sqrt(2.0 / np.pi) / np.log(2.0)
+_GELU_A = 0.044715 * _GELU_B
+
+
+def gelu_gate_ratios(c, h):
+    """Error of the epilogue's FP32 GELU against the float64 formula, as fractions of
+    the two gates the design's error analysis gives (both must stay <= 1):
+      gate 1: 2^-20 (|c| + |G|)   -- the analysis bounds the error by 2^-22.2 of it;
+      gate 2: 2^-20 |G| (1 + w |X|) + 2^-120, w = 2^X / (1 + 2^X): the relative error of
+              h, which grows with |X| where h is a small tail value (x = X(c) is formed
+              with three binary32 roundings, and h depends on 2^x; about 4 ln2 2^-24 |X|
+              w plus ~2^-21.4 from exp2, 1 + e, the reciprocal and the final product),
+              and an absolute floor below which the flush-to-zero reciprocal returns 0."""
+    c64 = c.astype(np.float64)
+    G = oracle.gelu_tanh(c)
+    X = c64 * (_GELU_A * c64 * c64 + _GELU_B)
+    w = 1.0 / (1.0 + np.exp2(np.minimum(-X, 1000.0)))
+    err = np.abs(h.astype(np.float64) - G)
+    g1 = 2.0 ** -20 * (np.abs(c64) + np.abs(G))
+    g2 = 2.0 ** -20 * np.abs(G) * (1.0 + w * np.abs(X)) + 2.0 ** -120
+    with np.errstate(divide="ignore", invalid="ignore"):
+        r1 = np.where(err == 0, 0.0, err / g1)
+        r2 = np.where(err == 0, 0.0, err / g2)
+    return r1, r2
+
+
 def test_fused_gelu_requant_epilogue(cuda_dev):
     M, N, K = 300, 512, 384
     c, h, q_h, g_h, amax_h, h_cal = fused_case(M, N, K, 24)
-    # (i) h is GELU(c) within 2^-16 (|c| + |h|) of the float64 formula (the epilogue's
-    # exp2/reciprocal hardware approximations stay below ~2^-17 relative)
-    ref_h = oracle.gelu_tanh(c)
-    err = np.abs(h.astype(np.float64) - ref_h)
-    assert np.all(err <= 2.0 ** -16 * (np.abs(c) + np.abs(ref_h)) + 1e-37)
+    # (i) h is GELU(c) within both gates of the FP32 evaluation's error analysis
+    r1, r2 = gelu_gate_ratios(c, h)
+    assert r1.max() <= 1.0 and r2.max() <= 1.0, (r1.max(), r2.max())
     assert np.array_equal(h, h_cal)  # deterministic
     # (ii) codes and scales are the oracle's quantization of the GPU's own h with the supplied g
     ref_q = oracle.quantize(h, gscale=g_h)
@@ -185,6 +211,30 @@ def test_fused_gelu_requant_epilogue(cuda_dev):
     assert np.all(raw[~used] == 0)
     # (iii) the reported amax is max|h|
     assert amax_h == float(np.abs(h).max())
+
+
+@pytest.mark.parametrize("M,N", [(512, 512), (128, 256)])  # CTA-pair kernel, single-CTA kernel
+def test_gelu_epilogue_tail_and_wide_range(cuda_dev, M, N):
+    """c spread over about [-14, 14] (A's tensor scale raised): the negative tail, where
+    GELU is a tiny value of c / 2^X, and the positive side where h -> c, both within
+    the two gates; h and C from the same call agree with the plain GEMM's c."""
+    K = 512
+    qx, _ = gpu_quantize(synth.activations(41, M, K), nv.SF_MMA)
+    qw, _ = gpu_quantize(synth.weights(41, 0, N, K), nv.SF_MMA)
+    c = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    nv.nvfp4_gemm(qx, qw, c)
+    qx.gscale.mul_(float(np.float32(14.0 / float(c.abs().max()))))
+    nv.nvfp4_gemm(qx, qw, c)
+    h = torch.empty((M, N), dtype=torch.float32, device="cuda")
+    nv.nvfp4_gemm(qx, qw, None, act=nv.ACT_GELU_TANH, h_out=h)
+    torch.cuda.synchronize()
+    cn, hn = c.cpu().numpy(), h.cpu().numpy()
+    assert np.count_nonzero((cn > -10) & (cn < -3)) >= 200
+    assert np.count_nonzero(cn > 6) >= 50
+    r1, r2 = gelu_gate_ratios(cn, hn)
+    print(f"GELU gate ratios M={M} N={N}: gate1 max {r1.max():.3f}, gate2 max {r2.max():.3f}")
+    assert r1.max() <= 1.0 and r2.max() <= 1.0, (r1.max(), r2.max())
+    assert device_status() == nv.OK
 
 
 @pytest.mark.slow
@@ -220,3 +270,49 @@ def test_fused_ffn_chunk_decomposed(cuda_dev):
     ref, bound = oracle.gemm_ref(codes, scales, g_h, c2, s2, g2, rows=rows)
     got = y.float().cpu().numpy()[rows].astype(np.float64)
     assert_within_bound(got, ref, bound, extra_rel=2.0 ** -8)
+
+
+@pytest.mark.slow
+def test_fused_ffn_end_to_end_vs_pure_oracle(cuda_dev):
+    """End-to-end report of the fused FFN chunk (X 8192 x 3072 -> 14336 with GELU and
+    NVFP4 requantization -> 3072, bf16) against a pure-oracle FFN on sampled rows:
+    oracle quantize of X, W1 and W2 -> float64 GEMM of the decoded operands -> FP32 c ->
+    float64 GELU -> FP32 h -> oracle quantize with the supplied tensor scale -> float64
+    GEMM.  GEMM1 is only bound-exact, so the GPU's h cannot match bit for bit: the
+    relative Frobenius error of the output and the mismatch rates of the intermediate's
+    codes and scales are printed (the numbers the design notes record) and held to a
+    loose sanity bound only.  The supplied scale is an input of the fused epilogue; both
+    sides get the same value, RN(max|h| / 2688) of the oracle's h on the sampled rows."""
+    M, K, N = 8192, 3072, 14336
+    x = synth.activations(4, M, K)
+    w1 = synth.weights(4, 0, N, K)
+    w2 = synth.weights(4, 1, K, N)
+    rows = np.arange(0, M, 257)
+    # ---- pure oracle
+    qx_o, q1_o, q2_o = oracle.quantize(x), oracle.quantize(w1), oracle.quantize(w2)
+    c_o, _ = oracle.gemm_ref(qx_o.codes, qx_o.scales, qx_o.g, q1_o.codes, q1_o.scales, q1_o.g, rows=rows)
+    h_o = oracle.gelu_tanh(c_o.astype(np.float32)).astype(np.float32)
+    g_h = float(np.float32(np.float32(np.abs(h_o).max()) / np.float32(2688.0)))
+    qh_o = oracle.quantize(h_o, gscale=g_h)
+    y_o, _ = oracle.gemm_ref(qh_o.codes, qh_o.scales, qh_o.g, q2_o.codes, q2_o.scales, q2_o.g)
+    # ---- GPU, through the C ABI
+    qx, _ = gpu_quantize(x, nv.SF_MMA)
+    q1, _ = gpu_quantize(w1, nv.SF_MMA)
+    q2, _ = gpu_quantize(w2, nv.SF_MMA)
+    q_h = nv.NVFP4Tensor(M, N, nv.SF_MMA)
+    nv.nvfp4_gemm(qx, q1, None, act=nv.ACT_GELU_TANH, q_out=q_h,
+                  q_gscale_in=torch.tensor([g_h], dtype=torch.float32, device="cuda"))
+    y = torch.empty((M, K), dtype=torch.bfloat16, device="cuda")
+    nv.nvfp4_gemm(q_h, q2, y)
+    torch.cuda.synchronize()
+    assert device_status() == nv.OK
+    y_g = y.float().cpu().numpy()[rows].astype(np.float64)
+    codes, scales, _ = canonical(q_h)
+    nib_g = np.stack([codes[rows] & 0xF, codes[rows] >> 4], axis=-1)
+    nib_o = np.stack([qh_o.codes & 0xF, qh_o.codes >> 4], axis=-1)
+    rel_fro = float(np.linalg.norm(y_g - y_o) / np.linalg.norm(y_o))
+    code_mis = float(np.mean(nib_g != nib_o))
+    scale_mis = float(np.mean(scales[rows] != qh_o.scales))
+    print(f"fused FFN vs pure-oracle FFN on {len(rows)} rows: relative Frobenius error {rel_fro:.3e}, "
+          f"code mismatch rate {code_mis:.3e}, scale mismatch rate {scale_mis:.3e}")
+    assert rel_fro < 1e-2 and code_mis < 1e-2 and scale_mis < 1e-2
