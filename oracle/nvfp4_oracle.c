@@ -362,10 +362,16 @@ void oracle_kv_dequant_chunk(const uint8_t* k_codes, const uint8_t* k_scales,
 
 /* ----------------------------------------------------------- activation */
 
-/* GELU, tanh form (Hendrycks & Gimpel), in double. */
+/* GELU, tanh form (Hendrycks & Gimpel), in double:
+ *   h = 0.5 c (1 + tanh(u)),  u = sqrt(2/pi) (c + 0.044715 c^3),
+ * evaluated through the exact identity 0.5 (1 + tanh(u)) = 1 / (1 + exp(-2u)), i.e.
+ * h = c / (1 + exp(-2u)).  Written as 1 + tanh(u), the sum cancels for u << 0 (tanh
+ * is -1 to within its rounding error), which leaves no correct digit in the negative
+ * tail; the quotient form keeps the relative error at a few ulp everywhere. */
 double oracle_gelu_tanh(double c) {
   const double k = sqrt(2.0 / 3.14159265358979323846);
-  return 0.5 * c * (1.0 + tanh(k * (c + 0.044715 * c * c * c)));
+  const double u = k * (c + 0.044715 * c * c * c);
+  return c / (1.0 + exp(-2.0 * u));
 }
 
 void oracle_gelu_tanh_array(const float* c, int64_t n, double* out) {
