@@ -95,6 +95,54 @@ __device__ __forceinline__ float rcp_approx(float x) {
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// ---------------------------------------------------------------- grid barrier
+__device__ __forceinline__ unsigned long long globaltimer_ns() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+constexpr unsigned long long kGridBarrierLimitNs = 2000000000ull;
+
+// Barrier of a whole grid whose CTAs are all resident at once (one wave, sized by
+// the occupancy query, launched after every earlier grid on the stream has
+// started).  *ctr is zero before the launch; each CTA adds one and waits for
+// gridDim.x arrivals.  The wait is bounded: false after limit_ns, and the caller
+// records a timeout instead of hanging.  Memory written by any CTA before the
+// barrier is visible to every CTA after it (release/acquire at GPU scope).
+__device__ __forceinline__ bool grid_barrier(unsigned* ctr, unsigned long long limit_ns) {
+  __shared__ int barrier_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    atomicAdd(ctr, 1u);
+    int ok = 1;
+    const unsigned long long t0 = globaltimer_ns();
+    while (ld_acquire_gpu(ctr) < gridDim.x) {
+      if (globaltimer_ns() - t0 > limit_ns) {
+        ok = 0;
+        break;
+      }
+      __nanosleep(100);
+    }
+    barrier_ok = ok;
+  }
+  __syncthreads();
+  return barrier_ok != 0;
+}
+
 // ---------------------------------------------------------------- E2M1
 // Exact E2M1 magnitude index of |x| / D by comparing |x| with each midpoint
 // m * D (m = 0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5).  fmaf gives the correctly

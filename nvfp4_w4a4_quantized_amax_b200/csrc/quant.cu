@@ -9,6 +9,8 @@
 //
 // Memory traffic per element (bf16 in): amax pass 2 B read; encode pass 2 B read,
 // 0.5 B codes + 1/16 B scale written.  Loads are 128-bit and read-only-path.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -79,6 +81,70 @@ struct EncodeParams {
   unsigned* status;
 };
 
+// The 16 values of virtual block vb (16 bf16 = 32 bytes, or 16 FP32 = 64 bytes).
+template <bool kBf16>
+__device__ __forceinline__ void load_block(const EncodeParams& p, uint32_t r, uint32_t j, float (&v)[16]) {
+  const uint8_t* src = p.x + (int64_t)r * p.x_row_bytes + (int64_t)j * (kBf16 ? 32 : 64);
+  if (kBf16) {
+    // the second load finds the other half of each 32-byte sector in L1
+    const uint4 a = ldg_nc_v4_l1(src), b = ldg_nc_v4_l1(src + 16);
+    const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      v[2 * k] = bf16_lo(w[k]);
+      v[2 * k + 1] = bf16_hi(w[k]);
+    }
+  } else {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const uint4 a = ldg_nc_v4_l1(src + 16 * k);
+      v[4 * k] = __uint_as_float(a.x);
+      v[4 * k + 1] = __uint_as_float(a.y);
+      v[4 * k + 2] = __uint_as_float(a.z);
+      v[4 * k + 3] = __uint_as_float(a.w);
+    }
+  }
+}
+
+// Encodes virtual block vb with tensor scale g (d6 = RN(6 g), r6 = RN(1 / d6)):
+// block amax -> E4M3 scale -> 16 codes.  Padding blocks of the tensor-core layout
+// get a zero scale.  local_max accumulates max|x| bits when `track` is set.
+template <bool kBf16, bool kMma>
+__device__ __forceinline__ void encode_block(const EncodeParams& p, int64_t vb, float g, float d6, float r6,
+                                             bool track, unsigned& local_max) {
+  const uint32_t r = p.vb_per_row.div((uint32_t)vb);
+  const uint32_t j = (uint32_t)vb - r * p.vb_per_row.d;
+  const int64_t soff = kMma ? sf_mma_offset(r, j, p.groups) : (int64_t)r * p.ld_scales + j;
+  if (kMma && (r >= p.rows || j >= p.nb)) {  // padding of the tensor-core layout
+    p.scales[soff] = 0;
+    return;
+  }
+  float v[16];
+  load_block<kBf16>(p, r, j, v);
+  float amax_b = 0.0f;
+#pragma unroll
+  for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(v[k]));
+  if (track) {
+    unsigned bits = 0;
+#pragma unroll
+    for (int k = 0; k < 16; ++k) bits = max(bits, __float_as_uint(v[k]) & 0x7FFFFFFFu);
+    local_max = max(local_max, bits);
+  }
+  const uint32_t s = block_scale_fast(amax_b, d6, r6);
+  const BlockEncoder enc(e4m3_to_float(s) * g);
+  float v0[8], v1[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    v0[k] = v[k];
+    v1[k] = v[8 + k];
+  }
+  uint2 out;
+  out.x = enc.encode8s(v0);
+  out.y = enc.encode8s(v1);
+  stg_v2(p.codes + (int64_t)r * p.ld_codes + (int64_t)j * 8, out);
+  p.scales[soff] = (uint8_t)s;
+}
+
 // One thread encodes one 16-value block: block amax -> E4M3 scale -> 16 codes.
 template <bool kBf16, bool kMma>
 __global__ void __launch_bounds__(kThreads) encode_kernel(EncodeParams p) {
@@ -104,65 +170,71 @@ __global__ void __launch_bounds__(kThreads) encode_kernel(EncodeParams p) {
   const float r6 = 1.0f / d6;
 
   unsigned local_max = 0;
+  const bool track = p.amax_accum != nullptr;
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   // Blocks are visited from the end of x backwards: the amax pass read x front to
   // back, so its most recent reads (still in L2) are encoded first.
-  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < p.nvblocks; i += stride) {
-    const int64_t vb = p.nvblocks - 1 - i;
-    const uint32_t r = p.vb_per_row.div((uint32_t)vb);
-    const uint32_t j = (uint32_t)vb - r * p.vb_per_row.d;
-    const int64_t soff = kMma ? sf_mma_offset(r, j, p.groups) : (int64_t)r * p.ld_scales + j;
-    if (kMma && (r >= p.rows || j >= p.nb)) {  // padding of the tensor-core layout
-      p.scales[soff] = 0;
-      continue;
-    }
-    float v[16];
-    const uint8_t* src = p.x + (int64_t)r * p.x_row_bytes + (int64_t)j * (kBf16 ? 32 : 64);
-    if (kBf16) {
-      // the second load finds the other half of each 32-byte sector in L1
-      const uint4 a = ldg_nc_v4_l1(src), b = ldg_nc_v4_l1(src + 16);
-      const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
-#pragma unroll
-      for (int k = 0; k < 8; ++k) {
-        v[2 * k] = bf16_lo(w[k]);
-        v[2 * k + 1] = bf16_hi(w[k]);
-      }
-    } else {
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint4 a = ldg_nc_v4_l1(src + 16 * k);
-        v[4 * k] = __uint_as_float(a.x);
-        v[4 * k + 1] = __uint_as_float(a.y);
-        v[4 * k + 2] = __uint_as_float(a.z);
-        v[4 * k + 3] = __uint_as_float(a.w);
-      }
-    }
-    float amax_b = 0.0f;
-#pragma unroll
-    for (int k = 0; k < 16; ++k) amax_b = fmaxf(amax_b, fabsf(v[k]));
-    if (p.amax_accum) {
-      unsigned bits = 0;
-#pragma unroll
-      for (int k = 0; k < 16; ++k) bits = max(bits, __float_as_uint(v[k]) & 0x7FFFFFFFu);
-      local_max = max(local_max, bits);
-    }
-    const uint32_t s = block_scale_fast(amax_b, d6, r6);
-    const BlockEncoder enc(e4m3_to_float(s) * g);
-    float v0[8], v1[8];
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      v0[k] = v[k];
-      v1[k] = v[8 + k];
-    }
-    uint2 out;
-    out.x = enc.encode8s(v0);
-    out.y = enc.encode8s(v1);
-    stg_v2(p.codes + (int64_t)r * p.ld_codes + (int64_t)j * 8, out);
-    p.scales[soff] = (uint8_t)s;
-  }
-  if (p.amax_accum) {
+  for (int64_t i = (int64_t)blockIdx.x * kThreads + threadIdx.x; i < p.nvblocks; i += stride)
+    encode_block<kBf16, kMma>(p, p.nvblocks - 1 - i, g, d6, r6, track, local_max);
+  if (track) {
     if (local_max >= 0x7F800000u) set_status(p.status, kStatusNonfinite);
     block_max_atomic(local_max, p.amax_accum);
+  }
+}
+
+// Grid-barrier counters of quantize_fused_kernel, one per launch slot: launches take
+// slots round robin and zero theirs on the stream first, so a slot is reused only
+// after kGridSyncSlots later launches (calls on other streams that overlap that many
+// launches would share a counter).
+constexpr int kGridSyncSlots = 256;
+__device__ unsigned g_grid_sync[kGridSyncSlots];
+
+// Quantization with an unknown tensor scale in ONE launch, for a tensor small
+// enough to stay in L2 between its two reads: every CTA takes the max|x| of its
+// blocks, the grid meets at a bounded barrier (all CTAs of the one-wave grid are
+// resident), then every CTA encodes the same blocks with g = RN(amax / 2688),
+// newest reads first, while they are still in L1/L2.  Replaces the zero + amax +
+// encode chain (two dependent launch boundaries) for such tensors; the result is
+// the same bits.  g_grid_sync[slot] is the grid-barrier counter, zeroed on the
+// stream before the launch.  The kernel lets its dependents start only once the whole grid has met,
+// so a dependent grid can never hold resources that one of its CTAs still needs.
+template <bool kBf16, bool kMma>
+__global__ void __launch_bounds__(kThreads) quantize_fused_kernel(EncodeParams p, unsigned* amax_bits,
+                                                                  int slot) {
+  pdl_wait();
+  const int64_t stride = (int64_t)gridDim.x * kThreads;
+  const int64_t first = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  unsigned m = 0;
+  for (int64_t vb = first; vb < p.nvblocks; vb += stride) {
+    const uint32_t r = p.vb_per_row.div((uint32_t)vb);
+    const uint32_t j = (uint32_t)vb - r * p.vb_per_row.d;
+    if (kMma && (r >= p.rows || j >= p.nb)) continue;
+    float v[16];
+    load_block<kBf16>(p, r, j, v);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) m = max(m, __float_as_uint(v[k]) & 0x7FFFFFFFu);
+  }
+  block_max_atomic(m, amax_bits);
+  if (!grid_barrier(&g_grid_sync[slot], kGridBarrierLimitNs)) {
+    if (threadIdx.x == 0) set_status(p.status, kStatusTimeout);
+    pdl_trigger();
+    return;
+  }
+  pdl_trigger();  // the whole grid is resident and past its first pass
+  const unsigned ab = ld_relaxed_gpu(amax_bits);
+  if (ab >= 0x7F800000u) {
+    if (blockIdx.x == 0 && threadIdx.x == 0) set_status(p.status, kStatusNonfinite);
+    return;
+  }
+  const float g = __uint_as_float(ab) / 2688.0f;
+  if (blockIdx.x == 0 && threadIdx.x == 0) *p.gscale_out = g;
+  const float d6 = 6.0f * g;
+  const float r6 = 1.0f / d6;
+  unsigned unused = 0;
+  if (first < p.nvblocks) {
+    const int64_t last = first + (p.nvblocks - 1 - first) / stride * stride;
+    for (int64_t vb = last; vb >= first; vb -= stride)
+      encode_block<kBf16, kMma>(p, vb, g, d6, r6, false, unused);
   }
 }
 
@@ -217,6 +289,12 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantParams p) {
   }
 }
 
+
+__global__ void zero_sync_kernel(unsigned* amax_bits, int slot) {
+  pdl_wait();
+  if (threadIdx.x == 0) *amax_bits = 0u;
+  if (threadIdx.x == 1) g_grid_sync[slot] = 0u;
+}
 
 // Zeroes n words before an accumulation: a kernel rather than a memset, so that
 // its launch overlaps the previous kernel.  It does not trigger its dependents
@@ -281,11 +359,30 @@ cudaError_t launch_amax(const QuantizeArgs& a, cudaStream_t s) {
   return launch_amax_pass(a.x, a.x_bf16, a.rows, a.cols, a.ldx, reinterpret_cast<unsigned*>(a.amax_out), s);
 }
 
+// Tensors up to this many bytes take the one-launch quantization (two reads of x
+// that stay in the 126 MB L2 between them; half of L2 leaves room for the outputs
+// and for what other kernels keep there).
+constexpr int64_t kFusedQuantizeMaxBytes = 64ll << 20;
+
+template <bool kBf16, bool kMma>
+static cudaError_t launch_fused(const EncodeParams& p, unsigned* amax_bits, cudaStream_t s) {
+  static std::atomic<unsigned> next_slot{0};
+  const int slot = (int)(next_slot.fetch_add(1, std::memory_order_relaxed) % kGridSyncSlots);
+  launch_pdl(zero_sync_kernel, 1, 32, 0, s, amax_bits, slot);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  // one wave: every CTA is resident at once, which the grid barrier needs
+  const int grid = wave_grid<quantize_fused_kernel<kBf16, kMma>>(kThreads, p.nvblocks);
+  launch_pdl(quantize_fused_kernel<kBf16, kMma>, grid, kThreads, 0, s, p, amax_bits, slot);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
   const int64_t esz = a.x_bf16 ? 2 : 4;
   const int64_t nb = a.cols / 16;
   unsigned* amax_bits = reinterpret_cast<unsigned*>(a.amax_out);
-  if (a.amax_out) {
+  const bool fused = !a.gscale_in && a.rows > 0 && a.rows * a.ldx * esz <= kFusedQuantizeMaxBytes;
+  if (a.amax_out && !fused) {
     cudaError_t e = launch_zero_words(a.amax_out, 1, s);
     if (e != cudaSuccess) return e;
   }
@@ -295,7 +392,7 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
     }
     return cudaMemcpyAsync(a.gscale_out, a.gscale_in, sizeof(float), cudaMemcpyDeviceToDevice, s);
   }
-  if (!a.gscale_in) {
+  if (!a.gscale_in && !fused) {
     cudaError_t e = launch_amax_pass(a.x, a.x_bf16, a.rows, a.cols, a.ldx, amax_bits, s);
     if (e != cudaSuccess) return e;
   }
@@ -318,6 +415,10 @@ cudaError_t launch_quantize(const QuantizeArgs& a, cudaStream_t s) {
   p.gscale_out = a.gscale_out;
   p.amax_accum = a.gscale_in ? amax_bits : nullptr;
   p.status = a.status;
+  if (fused) {
+    if (a.x_bf16) return a.sf_mma ? launch_fused<true, true>(p, amax_bits, s) : launch_fused<true, false>(p, amax_bits, s);
+    return a.sf_mma ? launch_fused<false, true>(p, amax_bits, s) : launch_fused<false, false>(p, amax_bits, s);
+  }
   const int64_t n = p.nvblocks;
   if (a.x_bf16) {
     if (a.sf_mma) launch_pdl(encode_kernel<true, true>, wave_grid<encode_kernel<true, true>>(kThreads, n), kThreads, 0, s, p);
