@@ -305,6 +305,32 @@ nvfp4_status kv_dequant_window_tokens(const nvfp4_kv_cache* cache, const int32_t
                                       const int32_t* tokens_host, int32_t n_slots, void* k_out,
                                       void* v_out, nvfp4_stream_t stream);
 
+/* kv_window_scores — attention scores of a block of queries against the keys of a
+ * window, reading K straight from the NVFP4 cache.  [TW] §四: the cache chunks of
+ * the attention window are dequantized together and feed attention; here the
+ * dequantization happens inside the kernel that computes Q K^T, one 128-key tile at
+ * a time in shared memory, so no bf16 copy of the window's K is written to HBM.
+ *   slots_host, tokens_host, n_slots : the window exactly as for
+ *              kv_dequant_window_tokens (HOST arrays); Tk = sum(tokens_host) keys,
+ *              in list order.
+ *   q        : device bf16 [tq][heads][head_dim], row pitch ldq elements
+ *              (ldq >= heads * head_dim); base and row pitch 16-byte aligned.
+ *   scale    : FP32 factor applied to every score (e.g. 1 / sqrt(head_dim)).
+ *   s_out    : device [heads][tq][ld_s] of st (NVFP4_FP32 or NVFP4_BF16), ld_s >= Tk,
+ *              base and row pitch 16-byte aligned:
+ *                S[h, i, j] = RN(scale * sum_d q[i, h, d] * K^[j, h, d]),
+ *              the sum accumulated in FP32 by the tensor cores (bf16 products are
+ *              exact), K^ bit for bit the window's K that kv_dequant_window_tokens
+ *              writes; bf16 output is the RNE of that value.  Columns j >= Tk are
+ *              not written.
+ * Requires head_dim == 128 (else NVFP4_ERR_SHAPE).  A listed slot whose recorded
+ * token count differs sets device status NVFP4_ERR_SHAPE; its scores are then
+ * unspecified.  Errors: INVALID_ARG (NULL, bad dtype or slot, non-finite scale),
+ * SHAPE, ALIGNMENT. */
+nvfp4_status kv_window_scores(const nvfp4_kv_cache* cache, const int32_t* slots_host, const int32_t* tokens_host,
+                              int32_t n_slots, const void* q, int64_t tq, int64_t ldq, float scale, void* s_out,
+                              int32_t st, int64_t ld_s, nvfp4_stream_t stream);
+
 /* ----------------------------------------------------------- amax history ----
  * A requantizing GEMM epilogue (nvfp4_epilogue.q_out) quantizes before its own
  * max|h| is known, so it takes a supplied tensor scale (q_gscale_in) and reports

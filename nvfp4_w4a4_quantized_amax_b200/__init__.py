@@ -67,6 +67,7 @@ class nvfp4_kv_cache(ctypes.Structure):
 EXPORTS = ["nvfp4_version", "nvfp4_status_string", "nvfp4_scales_bytes", "nvfp4_quantize", "nvfp4_amax",
            "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_cache_bytes", "nvfp4_kv_cache_init",
            "kv_quant_append", "kv_quant_append_noalloc", "kv_dequant_window", "kv_dequant_window_tokens",
+           "kv_window_scores",
            "nvfp4_lora_merge", "nvfp4_amax_history_push", "nvfp4_last_cuda_error_string",
            "nvfp4_debug_gemm_fault",
            "nvfp4_get_device_status"]
@@ -114,6 +115,9 @@ def library():
             lib.kv_dequant_window_tokens.restype = i32
             lib.kv_dequant_window_tokens.argtypes = [KV, ctypes.POINTER(ctypes.c_int32),
                                                      ctypes.POINTER(ctypes.c_int32), i32, vp, vp, vp]
+            lib.kv_window_scores.restype = i32
+            lib.kv_window_scores.argtypes = [KV, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), i32,
+                                             vp, i64, i64, ctypes.c_float, vp, i32, i64, vp]
             lib.nvfp4_lora_merge.restype = i32
             lib.nvfp4_lora_merge.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32, ctypes.c_float, vp, i64, vp]
             lib.nvfp4_amax_history_push.restype = i32
@@ -302,6 +306,20 @@ def kv_dequant_window_tokens(cache: KVCache, slots: Sequence[int], tokens: Seque
     tarr = (ctypes.c_int32 * len(tokens))(*tokens)
     _check(library().kv_dequant_window_tokens(ctypes.byref(cache.handle), sarr, tarr, len(slots), _ptr(k_out),
                                               _ptr(v_out), _stream(stream)), "kv_dequant_window_tokens")
+
+
+def kv_window_scores(cache: KVCache, slots: Sequence[int], tokens: Sequence[int], q, scale: float, s_out,
+                     stream=None):
+    """Scores of q (bf16 [tq, heads, head_dim]) against the window's keys, K read
+    from the NVFP4 cache inside the kernel; s_out (fp32 or bf16 [heads, tq, >= Tk])."""
+    if len(tokens) != len(slots):
+        raise ValueError("one token count per slot")
+    sarr = (ctypes.c_int32 * len(slots))(*slots)
+    tarr = (ctypes.c_int32 * len(tokens))(*tokens)
+    tq = q.shape[0]
+    _check(library().kv_window_scores(ctypes.byref(cache.handle), sarr, tarr, len(slots), _ptr(q), tq,
+                                      q.stride(0), float(scale), _ptr(s_out), _dtype_code(s_out),
+                                      s_out.stride(1), _stream(stream)), "kv_window_scores")
 
 
 def nvfp4_lora_merge(w, lora_b, lora_a, scale: float, out, stream=None):

@@ -20,8 +20,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(PKG, "libnvfp4.so")
-SOURCES = ["api.cu", "quant.cu", "kv.cu", "gemm.cu", "lora.cu"]
-HEADERS = ["common.cuh", "kernels.h"]
+SOURCES = ["api.cu", "quant.cu", "kv.cu", "gemm.cu", "lora.cu", "scores.cu"]
+HEADERS = ["common.cuh", "kernels.h", "tc.cuh"]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = [

@@ -112,6 +112,12 @@ constexpr int kMaxWindowSlots = 64;
 cudaError_t launch_kv_window(const KVLayout& c, const int32_t* slots, const int32_t* tokens, int32_t n_slots,
                              void* k_out, void* v_out, unsigned* status, cudaStream_t s);
 
+// Attention scores of q [tq][heads][128] (bf16, row pitch ldq elements) against the
+// window's keys, K dequantized from the cache inside the kernel; s_out [heads][tq][ld_s].
+cudaError_t launch_kv_scores(const KVLayout& c, const int32_t* slots, const int32_t* tokens, int32_t n_slots,
+                             const void* q, int64_t tq, int64_t ldq, float scale, void* s_out, bool s_bf16,
+                             int64_t ld_s, unsigned* status, cudaStream_t s);
+
 // Zero n_words 32-bit words of device memory (a PDL-launched kernel, not a memset).
 cudaError_t launch_zero_words(void* p, int n_words, cudaStream_t s);
 

@@ -1,0 +1,408 @@
+// scores.cu — attention scores straight from the NVFP4 KV cache.
+//
+// techwalker.com, "NVIDIA研究团队打造全球首个FP4视频生成系统，速度提升两倍还省一半内存", §四:
+// K and V are kept in NVFP4 (K after subtracting its mean) and the chunks of the
+// attention window are dequantized together.  Here the K side of that window is
+// consumed by the attention product itself: each CTA dequantizes one tile of 128
+// window keys of one head from the cache into shared memory (never to HBM), in the
+// tensor core's 128-byte-swizzled K-major layout, and multiplies every query tile of
+// that head with it on the tcgen05 tensor cores (kind::f16, bf16 x bf16, FP32
+// accumulators in tensor memory):
+//
+//   S[h, i, j] = RN(scale * sum_d Q[i, h, d] * K^[j, h, d])     (FP32 accumulate)
+//   K^[j, h, d] = bf16(RN(RN(e2m1 * s * g_K) + mu[h, d]))      (the window's K, bit for
+//                                                               bit what kv_dequant_window
+//                                                               writes)
+//
+// CTA (key tile kt, head h), 6 warps:
+//   all warps   dequantize the 128 x 128 K^ tile into shared memory (once per CTA)
+//   warp 0      TMA producer: query tiles (128 queries x 128 dims bf16, two 64-column
+//               boxes with the 128-byte swizzle), double-buffered
+//   warp 1      MMA issuer: 8 tcgen05.mma (K = 16 each) per query tile into one of two
+//               128-column accumulators in tensor memory
+//   warps 2..5  epilogue: one lane quarter each, tcgen05.ld of a query row's 128 scores,
+//               scaling, stores of the row's 128 keys (FP32 or bf16)
+// The dequantized keys are reused by every query tile, so the cache is read once per
+// (head, key tile) and no bf16 copy of the window exists in HBM.  Every wait is
+// bounded (2 s): a wait that gives up records NVFP4_ERR_TIMEOUT, the CTA drains its
+// own copies and MMAs and leaves.
+#include <atomic>
+#include <cstring>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tc.cuh"
+
+namespace nvfp4 {
+namespace {
+
+using namespace tc;
+
+constexpr int kQ = 128;          // queries per tile (MMA M, tensor-memory lanes)
+constexpr int kKeys = 128;       // keys per CTA (MMA N)
+constexpr int kD = 128;          // head_dim (MMA K, 8 instructions of 16)
+constexpr int kThreads = 192;    // 6 warps
+constexpr int kQBufs = 2;
+constexpr int kAcc = 2;
+constexpr int kKBytes = kKeys * kD * 2;  // 32 KB: two 128-row x 128-byte swizzled blocks
+constexpr int kQBytes = kQ * kD * 2;     // 32 KB
+constexpr int kBlockBytes = 128 * 128;   // one 64-column block of a 128-row tile
+constexpr int kSmemBytes = kKBytes + kQBufs * kQBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
+constexpr int kTmemCols = kAcc * kKeys;  // 256
+constexpr unsigned long long kWaitLimitNs = 2000000000ull;
+
+// kind::f16: D FP32 (bits 4..5 = 1), A and B bf16 (bits 7..9, 10..12 = 1), both
+// K-major, N >> 3 at bits 17..22, M >> 4 at bits 24..28.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kKeys >> 3) << 17) |
+                            ((uint32_t)(kQ >> 4) << 24);
+
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accumulate)
+      : "memory");
+}
+
+struct ScoresParams {
+  const uint8_t* base;
+  int64_t off_k_codes, off_k_scales, off_mu, off_gscale, off_tokens;
+  int64_t slot_codes_bytes, slot_scales_bytes;
+  int32_t heads, n_slots;
+  int32_t slots[kMaxWindowSlots];
+  int32_t tokens[kMaxWindowSlots];
+  int64_t key_end[kMaxWindowSlots];  // cumulative window keys through list entry i
+  int64_t Tq, Tk;
+  float scale;
+  uint8_t* s_out;
+  bool s_bf16;
+  int64_t ld_s;          // elements between query rows of one head
+  int64_t head_stride;   // elements between heads (Tq * ld_s)
+  unsigned* status;
+  unsigned long long wait_limit_ns;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    kv_scores_kernel(const __grid_constant__ CUtensorMap map_q, ScoresParams p) {
+  pdl_trigger();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* kbuf = smem;                  // K^ tile, 1024-aligned
+  uint8_t* qbuf = smem + kKBytes;        // kQBufs query tiles
+  uint8_t* bar_area = qbuf + kQBufs * kQBytes;
+  uint64_t* q_full = reinterpret_cast<uint64_t*>(bar_area);
+  uint64_t* q_empty = q_full + kQBufs;
+  uint64_t* t_full = q_empty + kQBufs;
+  uint64_t* t_empty = t_full + kAcc;
+  uint64_t* done_bar = t_empty + kAcc;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  __shared__ int32_t row_slot[kKeys];    // per key row: cache slot (-1: none)
+  __shared__ int32_t row_token[kKeys];   // token within the slot
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kt = blockIdx.x, h = blockIdx.y;
+  const int64_t n_qt = (p.Tq + kQ - 1) / kQ;
+  const unsigned long long limit = p.wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < kQBufs; ++b) {
+      mbar_init(smem_u32(&q_full[b]), 1);
+      mbar_init(smem_u32(&q_empty[b]), 1);
+    }
+    for (int a = 0; a < kAcc; ++a) {
+      mbar_init(smem_u32(&t_full[a]), 1);
+      mbar_init(smem_u32(&t_empty[a]), 4);
+    }
+    mbar_init(smem_u32(done_bar), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the cache, the queries and the output buffer come from earlier work
+
+  // the first query tiles load while the keys are dequantized
+  uint32_t issued = 0;
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_q)) : "memory");
+    for (; issued < (uint32_t)min((int64_t)kQBufs, n_qt); ++issued) {
+      const uint32_t fb = smem_u32(&q_full[issued]);
+      mbar_arrive_expect_tx(fb, kQBytes);
+      uint8_t* dst = qbuf + issued * kQBytes;
+      tma_load_2d(smem_u32(dst), &map_q, fb, h * kD, (int32_t)(issued * kQ));
+      tma_load_2d(smem_u32(dst + kBlockBytes), &map_q, fb, h * kD + 64, (int32_t)(issued * kQ));
+    }
+  }
+
+  // ---- the key tile: window position -> (slot, token), then K^ into shared memory
+  if (threadIdx.x < kKeys) {
+    const int64_t j = (int64_t)kt * kKeys + threadIdx.x;
+    int32_t sl = -1, tk = 0;
+    if (j < p.Tk) {
+      int i = 0;
+      while (j >= p.key_end[i]) ++i;
+      const int64_t begin = i == 0 ? 0 : p.key_end[i - 1];
+      const int32_t slot = p.slots[i];
+      const bool ok = reinterpret_cast<const int32_t*>(p.base + p.off_tokens)[slot] == p.tokens[i];
+      if (ok) {
+        sl = slot;
+        tk = (int32_t)(j - begin);
+      } else if (j == begin || threadIdx.x == 0) {
+        set_status(p.status, kStatusShape);  // the slot holds another token count
+      }
+    }
+    row_slot[threadIdx.x] = sl;
+    row_token[threadIdx.x] = tk;
+  }
+  __syncthreads();
+  const int64_t C = (int64_t)p.heads * kD;
+  for (int ci = threadIdx.x; ci < kKeys * kD / 8; ci += kThreads) {
+    const int r = ci >> 4, c16 = ci & 15;  // key row, 8-value chunk along head_dim
+    const int d0 = c16 * 8;
+    uint4 out = make_uint4(0, 0, 0, 0);
+    const int32_t slot = row_slot[r];
+    if (slot >= 0) {
+      const int64_t e = ((int64_t)row_token[r] * p.heads + h) * kD + d0;  // element within the slot
+      const uint32_t kc = *reinterpret_cast<const uint32_t*>(p.base + p.off_k_codes + slot * p.slot_codes_bytes + e / 2);
+      const uint32_t ks2 = e4m3_to_f16x2_bcast(p.base[p.off_k_scales + slot * p.slot_scales_bytes + e / 16]);
+      const float gk = reinterpret_cast<const float*>(p.base + p.off_gscale)[2 * slot];
+      const float4* m4 = reinterpret_cast<const float4*>(p.base + p.off_mu + ((int64_t)slot * C + h * kD + d0) * 4);
+      const float4 m0 = m4[0], m1 = m4[1];
+      const float mu[8] = {m0.x, m0.y, m0.z, m0.w, m1.x, m1.y, m1.z, m1.w};
+      uint32_t kh[4];
+      e2m1x8_times_scale(kc, ks2, kh);
+      float ko[8];
+#pragma unroll
+      for (int q = 0; q < 4; ++q) f16x2_to_f32x2(kh[q], ko[2 * q], ko[2 * q + 1]);  // e2m1 * s, exact
+#pragma unroll
+      for (int q = 0; q < 8; ++q) ko[q] = ko[q] * gk + mu[q];  // two roundings: -fmad=false
+      out = make_uint4(pack_bf16x2(ko[0], ko[1]), pack_bf16x2(ko[2], ko[3]), pack_bf16x2(ko[4], ko[5]),
+                       pack_bf16x2(ko[6], ko[7]));
+    }
+    // 128-byte swizzle: 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+    const int blk = d0 >> 6, c = (d0 & 63) >> 3;
+    *reinterpret_cast<uint4*>(kbuf + blk * kBlockBytes + r * 128 + ((c ^ (r & 7)) << 4)) = out;
+  }
+  fence_proxy_async_smem();  // the tensor core reads K^ through the async proxy
+  __syncthreads();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      bool ok = true;
+      for (uint32_t qt = issued; qt < (uint32_t)n_qt; ++qt) {
+        const int b = qt % kQBufs;
+        const uint32_t ph = (qt / kQBufs) & 1u;
+        if (!mbar_wait(smem_u32(&q_empty[b]), ph ^ 1u, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = smem_u32(&q_full[b]);
+        mbar_arrive_expect_tx(fb, kQBytes);
+        uint8_t* dst = qbuf + b * kQBytes;
+        tma_load_2d(smem_u32(dst), &map_q, fb, h * kD, (int32_t)(qt * kQ));
+        tma_load_2d(smem_u32(dst + kBlockBytes), &map_q, fb, h * kD + 64, (int32_t)(qt * kQ));
+        issued = qt + 1;
+      }
+      if (!ok) {
+        set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+      for (uint32_t j = issued > (uint32_t)kQBufs ? issued - kQBufs : 0; j < issued; ++j)
+        mbar_wait_drain(smem_u32(&q_full[j % kQBufs]), (j / kQBufs) & 1u, limit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      const uint32_t k_addr = smem_u32(kbuf);
+      for (uint32_t qt = 0; qt < (uint32_t)n_qt; ++qt) {
+        const int b = qt % kQBufs, a = qt % kAcc;
+        if (!mbar_wait(smem_u32(&t_empty[a]), ((qt / kAcc) & 1u) ^ 1u, abort_flag, limit) ||
+            !mbar_wait(smem_u32(&q_full[b]), (qt / kQBufs) & 1u, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        const uint32_t q_addr = smem_u32(qbuf + b * kQBytes);
+        const uint32_t d_tmem = tmem_base + a * kKeys;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          // K = 16 bf16 = 32 bytes of each swizzled 128-byte row: 4 per 64-column block
+          const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
+          mma_bf16(d_tmem, smem_desc(q_addr + off, 16, 1024, 2), smem_desc(k_addr + off, 16, 1024, 2),
+                   kk > 0 ? 1u : 0u);
+        }
+        commit(smem_u32(&q_empty[b]));
+        commit(smem_u32(&t_full[a]));
+      }
+      if (!ok) {
+        set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+      commit(smem_u32(done_bar));
+      mbar_wait_drain(smem_u32(done_bar), 0, limit);
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int quarter = warp & 3;  // the tensor-memory lanes this warp may access
+    const int64_t key0 = (int64_t)kt * kKeys;
+    const int nkeys = (int)min((int64_t)kKeys, p.Tk - key0);
+    for (uint32_t qt = 0; qt < (uint32_t)n_qt; ++qt) {
+      const int a = qt % kAcc;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&t_full[a]), (qt / kAcc) & 1u, abort_flag, limit))) {
+        if (lane == 0) set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+        break;
+      }
+      fence_after();
+      const int64_t qrow = (int64_t)qt * kQ + quarter * 32 + lane;
+      uint8_t* dst = p.s_out + ((int64_t)h * p.head_stride + qrow * p.ld_s + key0) * (p.s_bf16 ? 2 : 4);
+#pragma unroll 1
+      for (int cc = 0; cc < kKeys; cc += 32) {
+        uint32_t r[32];
+        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + a * kKeys + cc, r);
+        __syncwarp();
+        if (qrow >= p.Tq || cc >= nkeys) continue;  // no warp-collective work follows in this pass
+        float v[32];
+#pragma unroll
+        for (int i = 0; i < 32; i += 2)
+          mul2(v[i], v[i + 1], __uint_as_float(r[i]), __uint_as_float(r[i + 1]), p.scale, p.scale);
+        const int nv = min(32, nkeys - cc);  // a multiple of 8 unless the window ends here
+        if (p.s_bf16) {
+          uint8_t* d = dst + cc * 2;
+          if (nv == 32) {
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              stg_v4(d + 16 * u, make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
+                                            pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
+                                            pack_bf16x2(v[8 * u + 6], v[8 * u + 7])));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < nv) reinterpret_cast<uint16_t*>(d)[i] = (uint16_t)(pack_bf16x2(v[i], 0.0f) & 0xFFFFu);
+          }
+        } else {
+          float* d = reinterpret_cast<float*>(dst) + cc;
+          if (nv == 32) {
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              stg_v4(d + 4 * u, make_uint4(__float_as_uint(v[4 * u]), __float_as_uint(v[4 * u + 1]),
+                                           __float_as_uint(v[4 * u + 2]), __float_as_uint(v[4 * u + 3])));
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if (i < nv) d[i] = v[i];
+          }
+        }
+      }
+      fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&t_empty[a]));
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 0) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static std::atomic<EncodeTiledFn> cached{nullptr};
+  EncodeTiledFn fn = cached.load(std::memory_order_relaxed);
+  if (!fn) {
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess) {
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+      cached.store(fn, std::memory_order_relaxed);
+    }
+  }
+  return fn;
+}
+
+}  // namespace
+
+cudaError_t launch_kv_scores(const KVLayout& L, const int32_t* slots, const int32_t* tokens, int32_t n_slots,
+                             const void* q, int64_t tq, int64_t ldq, float scale, void* s_out, bool s_bf16,
+                             int64_t ld_s, unsigned* status, cudaStream_t s) {
+  if (L.head_dim != kD) return cudaErrorInvalidValue;
+  ScoresParams p;
+  memset(&p, 0, sizeof(p));
+  p.base = L.base;
+  p.off_k_codes = L.off_k_codes;
+  p.off_k_scales = L.off_k_scales;
+  p.off_mu = L.off_mu;
+  p.off_gscale = L.off_gscale;
+  p.off_tokens = L.off_tokens;
+  p.slot_codes_bytes = L.slot_codes_bytes;
+  p.slot_scales_bytes = L.slot_scales_bytes;
+  p.heads = L.heads;
+  p.n_slots = n_slots;
+  int64_t acc = 0;
+  for (int i = 0; i < n_slots; ++i) {
+    p.slots[i] = slots[i];
+    p.tokens[i] = tokens[i];
+    acc += tokens[i];
+    p.key_end[i] = acc;
+  }
+  p.Tq = tq;
+  p.Tk = acc;
+  p.scale = scale;
+  p.s_out = static_cast<uint8_t*>(s_out);
+  p.s_bf16 = s_bf16;
+  p.ld_s = ld_s;
+  p.head_stride = tq * ld_s;
+  p.status = status;
+  p.wait_limit_ns = kWaitLimitNs;
+  if (tq == 0) return cudaSuccess;
+
+  // queries [tq][heads * 128] bf16 (row pitch ldq elements): 64-column x 128-row boxes
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorInvalidValue;
+  CUtensorMap mq;
+  cuuint64_t dims[2] = {(cuuint64_t)L.heads * kD, (cuuint64_t)tq};
+  cuuint64_t strides[1] = {(cuuint64_t)ldq * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)kQ};
+  cuuint32_t estr[2] = {1, 1};
+  if (fn(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(q), dims, strides, box, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
+  static std::atomic<bool> done[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!done[dev].load(std::memory_order_relaxed)) {
+    e = cudaFuncSetAttribute(kv_scores_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
+    if (e != cudaSuccess) return e;
+    done[dev].store(true, std::memory_order_relaxed);
+  }
+  const dim3 grid((unsigned)((acc + kKeys - 1) / kKeys), (unsigned)L.heads, 1);
+  launch_pdl(kv_scores_kernel, grid, kThreads, kSmemBytes, s, mq, p);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4
