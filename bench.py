@@ -42,6 +42,7 @@ HEADS, HEAD_DIM, CHUNK, SLOTS, WINDOW = 24, 128, 8192, 16, 4
 ACT_ROWS, ACT_COLS = 32768, 3072
 BLOCK_GEMMS = [(3072, 3072), (3072, 9216), (3072, 14336), (14336, 3072)]  # (K, N)
 FFN = (3072, 14336)
+SCORES_TQ = 1024  # queries scored against the 4-chunk window by the attention-side consumer
 METRIC = "W4A4 GEMM TFLOPS; NVFP4 quant/KV-dequant GB/s; % of B200 roofline"
 WORKLOAD = ("longlive_dit_block_chunk: act quant/dequant 32768x3072; GEMMs M=8192 "
             "(3072->3072, 3072->9216, 3072->14336, 14336->3072); KV 24x128 append 8192 tok + "
@@ -371,10 +372,62 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     if status != nv.OK:
         raise RuntimeError("device status: " + nv.status_string(status))
 
+    # ---- the attention-side consumer of the cache (a "next" row, outside the step):
+    # scores of SCORES_TQ queries against the latest 4-chunk window with K read from
+    # the NVFP4 cache inside the kernel, against the window dequant to bf16 followed
+    # by a bf16 batched GEMM (cuBLAS through torch.bmm) on the dequantized keys
+    win = [(slot_counter[0] - WINDOW + j) % SLOTS for j in range(WINDOW)]
+    q = to_dev(synth.activations(5 + seed_off, SCORES_TQ, HEADS * HEAD_DIM)).view(SCORES_TQ, HEADS, HEAD_DIM)
+    s_fused = torch.empty((HEADS, SCORES_TQ, WINDOW * CHUNK), dtype=torch.bfloat16, device=dev)
+    s_pair = torch.empty_like(s_fused)
+    ko, vo = outs[0].ko, outs[0].vo
+
+    def fused():
+        nv.kv_window_scores(cache, win, [CHUNK] * WINDOW, q, 1.0, s_fused)
+
+    def pair():
+        nv.kv_dequant_window(cache, win, ko, vo)
+        torch.bmm(q.transpose(0, 1), ko.permute(1, 2, 0), out=s_pair)
+
+    scores = {}
+    for name, fn in (("kv_window_scores", fused), ("window_then_bmm", pair)):
+        for _ in range(3):
+            fn()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(10):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        scores[name] = e0.elapsed_time(e1) / 10
+    del s_fused, s_pair
+    status = nv.get_device_status(local_rank)
+    if status != nv.OK:
+        raise RuntimeError("device status: " + nv.status_string(status))
+
     # ---- max over ranks
     ms_per_step, e2e_ms = max_over_ranks([elapsed_ms / args.steps, e2e_ms], dist, dev)
     return {"ms_per_step": ms_per_step, "e2e_ms": e2e_ms, "kernels": kernels, "clocks": clocks,
-            "launches": n_launch, "h2d": h2d, "d2h": d2h}
+            "launches": n_launch, "h2d": h2d, "d2h": d2h, "scores": scores}
+
+
+def scores_summary(t, peaks):
+    """Scores of SCORES_TQ queries x 24 heads against the 32768-key window, bf16 out:
+    algorithmic bytes = K codes and scales read + queries read + scores written."""
+    keys = WINDOW * CHUNK
+    c = HEADS * HEAD_DIM
+    fused_bytes = keys * c // 2 + keys * c // 16 + SCORES_TQ * c * 2 + HEADS * SCORES_TQ * keys * 2
+    pair_bytes = (WINDOW * 2 * (CHUNK * c // 2 + CHUNK * c // 16) + WINDOW * 2 * 2 * CHUNK * c  # window
+                  + keys * c * 2 + SCORES_TQ * c * 2 + HEADS * SCORES_TQ * keys * 2)             # bmm
+    gbs = fused_bytes / (t["kv_window_scores"] * 1e-3) / 1e9
+    return {"workload": f"{SCORES_TQ} queries x {HEADS} heads x 128 against {keys} window keys, bf16 scores",
+            "kv_window_scores_ms": round(t["kv_window_scores"], 4),
+            "window_then_bmm_ms": round(t["window_then_bmm"], 4),
+            "speedup": round(t["window_then_bmm"] / t["kv_window_scores"], 3),
+            "fused_alg_bytes": fused_bytes, "pair_alg_bytes": pair_bytes,
+            "fused_gbs": round(gbs, 1), "fused_frac_hbm": round(gbs / peaks["hbm_gbs"], 3),
+            "flops": 2.0 * HEADS * SCORES_TQ * keys * HEAD_DIM}
 
 
 # Datasheet figures of one B200 (dense, no sparsity), reported beside the measured ones.
@@ -458,6 +511,7 @@ def summarize(res, args, world):
                 "d2h_bytes_per_step": res["d2h"]},
         "gpu_launches": res["launches"],
         "clocks": res["clocks"],
+        "next_rows": {"attention_side_dequant": scores_summary(res["scores"], peaks)},
     }
 
 
@@ -686,6 +740,18 @@ def run_single_kernel(args):
         ko = torch.empty((sum(fills), HEADS, HEAD_DIM), dtype=torch.bfloat16, device=dev)
         vo = torch.empty_like(ko)
         fn = lambda: nv.kv_dequant_window_tokens(cache, list(range(6)), fills, ko, vo)  # noqa: E731
+    elif args.kernel == "kv_scores":
+        # attention scores of 256 queries x 24 heads against a 4-chunk window, bf16 out
+        off = synth.kv_offsets(3, HEADS, HEAD_DIM)
+        k, v = synth.kv_chunk(3, 0, CHUNK, HEADS, HEAD_DIM, off)
+        kd, vd = to_dev(k), to_dev(v)
+        cache = nv.KVCache(HEADS, HEAD_DIM, CHUNK, WINDOW, dev)
+        for sl in range(WINDOW):
+            nv.kv_quant_append(cache, kd, vd, sl)
+        tq = 256
+        q = to_dev(synth.activations(5, tq, HEADS * HEAD_DIM)).view(tq, HEADS, HEAD_DIM)
+        s_out = torch.empty((HEADS, tq, WINDOW * CHUNK), dtype=torch.bfloat16, device=dev)
+        fn = lambda: nv.kv_window_scores(cache, list(range(WINDOW)), [CHUNK] * WINDOW, q, 1.0, s_out)  # noqa: E731
     elif args.kernel in ("kv_append", "kv_window"):
         off = synth.kv_offsets(3, HEADS, HEAD_DIM)
         k, v = synth.kv_chunk(3, 0, CHUNK, HEADS, HEAD_DIM, off)
@@ -750,7 +816,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel", default=None,
-                    help="profiling mode: gemm | gemm_fused | quantize | dequantize | kv_append | kv_window | kv_window_sink | lora_merge")
+                    help="profiling mode: gemm | gemm_fused | quantize | dequantize | kv_append | kv_window | kv_window_sink | "
+                         "kv_scores | lora_merge")
     ap.add_argument("--shape", default="8192,14336,3072", help="M,N,K for gemm; rows,cols for (de)quantize")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--kernel-warmup", type=int, default=1,
