@@ -321,8 +321,10 @@ nvfp4_status kv_dequant_window_tokens(const nvfp4_kv_cache* cache, const int32_t
  *                S[h, i, j] = RN(scale * sum_d q[i, h, d] * K^[j, h, d]),
  *              the sum accumulated in FP32 by the tensor cores (bf16 products are
  *              exact), K^ bit for bit the window's K that kv_dequant_window_tokens
- *              writes; bf16 output is the RNE of that value.  Columns j >= Tk are
- *              not written.
+ *              writes; bf16 output is the RNE of that value.  Each row is written
+ *              in whole 16-byte units: its elements from Tk up to the next 16-byte
+ *              boundary receive 0 (inside the row, since ld_s * size is a multiple
+ *              of 16); elements beyond that boundary are not written.
  * Requires head_dim == 128 (else NVFP4_ERR_SHAPE).  A listed slot whose recorded
  * token count differs sets device status NVFP4_ERR_SHAPE; its scores are then
  * unspecified.  Errors: INVALID_ARG (NULL, bad dtype or slot, non-finite scale),

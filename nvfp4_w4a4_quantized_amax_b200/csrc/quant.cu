@@ -190,30 +190,40 @@ constexpr int kGridSyncSlots = 256;
 __device__ unsigned g_grid_sync[kGridSyncSlots];
 
 // Quantization with an unknown tensor scale in ONE launch, for a tensor small
-// enough to stay in L2 between its two reads: every CTA takes the max|x| of its
-// blocks, the grid meets at a bounded barrier (all CTAs of the one-wave grid are
-// resident), then every CTA encodes the same blocks with g = RN(amax / 2688),
-// newest reads first, while they are still in L1/L2.  Replaces the zero + amax +
-// encode chain (two dependent launch boundaries) for such tensors; the result is
-// the same bits.  g_grid_sync[slot] is the grid-barrier counter, zeroed on the
-// stream before the launch.  The kernel lets its dependents start only once the whole grid has met,
-// so a dependent grid can never hold resources that one of its CTAs still needs.
+// enough to stay in L2 between its two reads: every CTA takes max|x| over a
+// grid-stride share of x, the grid meets at a bounded barrier (all CTAs of the
+// one-wave grid are resident), then every CTA encodes its blocks with
+// g = RN(amax / 2688) while x is still in L2.  Replaces the zero + amax + encode
+// chain (two dependent launch boundaries) for such tensors; the result is the same
+// bits.  g_grid_sync[slot] is the grid-barrier counter, zeroed on the stream before
+// the launch.  The kernel lets its dependents start only once the whole grid has
+// met, so a dependent grid can never hold resources that one of its CTAs still needs.
 template <bool kBf16, bool kMma>
 __global__ void __launch_bounds__(kThreads) quantize_fused_kernel(EncodeParams p, unsigned* amax_bits,
-                                                                  int slot) {
+                                                                  int slot, int64_t nchunks, FastDiv cpr) {
   pdl_wait();
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   const int64_t first = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+  // first pass: max|x| with one coalesced 16-byte load per thread and step (the
+  // layout of the amax kernel); x lands in L2 for the second pass
   unsigned m = 0;
-  for (int64_t vb = first; vb < p.nvblocks; vb += stride) {
-    const uint32_t r = p.vb_per_row.div((uint32_t)vb);
-    const uint32_t j = (uint32_t)vb - r * p.vb_per_row.d;
-    if (kMma && (r >= p.rows || j >= p.nb)) continue;
-    float v[16];
-    load_block<kBf16>(p, r, j, v);
-#pragma unroll
-    for (int k = 0; k < 16; ++k) m = max(m, __float_as_uint(v[k]) & 0x7FFFFFFFu);
+  for (int64_t i = first; i < nchunks; i += stride) {
+    const uint32_t r = cpr.div((uint32_t)i);
+    const uint32_t c = (uint32_t)i - r * cpr.d;
+    const uint4 v = ldg_nc_v4(p.x + (int64_t)r * p.x_row_bytes + (int64_t)c * 16);
+    if (kBf16) {
+      m = __vmaxu2(m, v.x & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.y & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.z & 0x7FFF7FFFu);
+      m = __vmaxu2(m, v.w & 0x7FFF7FFFu);
+    } else {
+      m = max(m, v.x & 0x7FFFFFFFu);
+      m = max(m, v.y & 0x7FFFFFFFu);
+      m = max(m, v.z & 0x7FFFFFFFu);
+      m = max(m, v.w & 0x7FFFFFFFu);
+    }
   }
+  if (kBf16) m = max(m >> 16, m & 0xFFFFu) << 16;
   block_max_atomic(m, amax_bits);
   if (!grid_barrier(&g_grid_sync[slot], kGridBarrierLimitNs)) {
     if (threadIdx.x == 0) set_status(p.status, kStatusTimeout);
@@ -231,11 +241,10 @@ __global__ void __launch_bounds__(kThreads) quantize_fused_kernel(EncodeParams p
   const float d6 = 6.0f * g;
   const float r6 = 1.0f / d6;
   unsigned unused = 0;
-  if (first < p.nvblocks) {
-    const int64_t last = first + (p.nvblocks - 1 - first) / stride * stride;
-    for (int64_t vb = last; vb >= first; vb -= stride)
-      encode_block<kBf16, kMma>(p, vb, g, d6, r6, false, unused);
-  }
+  // second pass from the end backwards: the first pass's latest reads are the most
+  // likely still in L2
+  for (int64_t i = first; i < p.nvblocks; i += stride)
+    encode_block<kBf16, kMma>(p, p.nvblocks - 1 - i, g, d6, r6, false, unused);
 }
 
 struct DequantParams {
@@ -373,7 +382,9 @@ static cudaError_t launch_fused(const EncodeParams& p, unsigned* amax_bits, cuda
   if (e != cudaSuccess) return e;
   // one wave: every CTA is resident at once, which the grid barrier needs
   const int grid = wave_grid<quantize_fused_kernel<kBf16, kMma>>(kThreads, p.nvblocks);
-  launch_pdl(quantize_fused_kernel<kBf16, kMma>, grid, kThreads, 0, s, p, amax_bits, slot);
+  const int64_t cpr = p.nb * (kBf16 ? 2 : 4);  // 16-byte chunks of x per row
+  launch_pdl(quantize_fused_kernel<kBf16, kMma>, grid, kThreads, 0, s, p, amax_bits, slot, p.rows * cpr,
+             FastDiv((uint32_t)cpr));
   return cudaGetLastError();
 }
 

@@ -17,11 +17,13 @@
 // CTA (key tile kt, head h), 6 warps:
 //   all warps   dequantize the 128 x 128 K^ tile into shared memory (once per CTA)
 //   warp 0      TMA producer: query tiles (128 queries x 128 dims bf16, two 64-column
-//               boxes with the 128-byte swizzle), double-buffered
+//               boxes with the 128-byte swizzle); two CTAs per SM overlap each other
 //   warp 1      MMA issuer: 8 tcgen05.mma (K = 16 each) per query tile into one of two
 //               128-column accumulators in tensor memory
 //   warps 2..5  epilogue: one lane quarter each, tcgen05.ld of a query row's 128 scores,
-//               scaling, stores of the row's 128 keys (FP32 or bf16)
+//               scaling, 32-row x 128-byte boxes staged in shared memory (128-byte
+//               swizzle) and written by TMA stores clipped to the head's queries and
+//               the window's keys
 // The dequantized keys are reused by every query tile, so the cache is read once per
 // (head, key tile) and no bf16 copy of the window exists in HBM.  Every wait is
 // bounded (2 s): a wait that gives up records NVFP4_ERR_TIMEOUT, the CTA drains its
@@ -42,12 +44,15 @@ constexpr int kQ = 128;          // queries per tile (MMA M, tensor-memory lanes
 constexpr int kKeys = 128;       // keys per CTA (MMA N)
 constexpr int kD = 128;          // head_dim (MMA K, 8 instructions of 16)
 constexpr int kThreads = 192;    // 6 warps
-constexpr int kQBufs = 2;
+constexpr int kQBufs = 1;          // two CTAs share an SM: one overlaps the other's query loads
 constexpr int kAcc = 2;
 constexpr int kKBytes = kKeys * kD * 2;  // 32 KB: two 128-row x 128-byte swizzled blocks
 constexpr int kQBytes = kQ * kD * 2;     // 32 KB
 constexpr int kBlockBytes = 128 * 128;   // one 64-column block of a 128-row tile
-constexpr int kSmemBytes = kKBytes + kQBufs * kQBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
+constexpr int kBoxBytes = 32 * 128;      // one output box: 32 query rows x 128 bytes
+constexpr int kStageBytes = 4 * 2 * kBoxBytes;  // two boxes in flight per epilogue warp
+constexpr int kSmemBytes = kKBytes + kQBufs * kQBytes + kStageBytes + 1024 /*barriers*/ + 1024 /*alignment*/;
+constexpr int kChunksPerThread = (kKeys * kD / 8 + kThreads - 1) / kThreads;  // 8-value chunks of K^
 constexpr int kTmemCols = kAcc * kKeys;  // 256
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 
@@ -75,22 +80,21 @@ struct ScoresParams {
   int64_t key_end[kMaxWindowSlots];  // cumulative window keys through list entry i
   int64_t Tq, Tk;
   float scale;
-  uint8_t* s_out;
   bool s_bf16;
-  int64_t ld_s;          // elements between query rows of one head
-  int64_t head_stride;   // elements between heads (Tq * ld_s)
   unsigned* status;
   unsigned long long wait_limit_ns;
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-    kv_scores_kernel(const __grid_constant__ CUtensorMap map_q, ScoresParams p) {
+    kv_scores_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_s,
+                     ScoresParams p) {
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* kbuf = smem;                  // K^ tile, 1024-aligned
   uint8_t* qbuf = smem + kKBytes;        // kQBufs query tiles
-  uint8_t* bar_area = qbuf + kQBufs * kQBytes;
+  uint8_t* stage = qbuf + kQBufs * kQBytes;  // output boxes, 8 KB per epilogue warp
+  uint8_t* bar_area = stage + kStageBytes;
   uint64_t* q_full = reinterpret_cast<uint64_t*>(bar_area);
   uint64_t* q_empty = q_full + kQBufs;
   uint64_t* t_full = q_empty + kQBufs;
@@ -166,15 +170,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   __syncthreads();
   const int64_t C = (int64_t)p.heads * kD;
-  for (int ci = threadIdx.x; ci < kKeys * kD / 8; ci += kThreads) {
+  // every code word and scale byte of this thread's chunks in flight at once
+  uint32_t kcw[kChunksPerThread], ksb[kChunksPerThread];
+#pragma unroll
+  for (int u = 0; u < kChunksPerThread; ++u) {
+    const int ci = threadIdx.x + u * kThreads;
+    kcw[u] = 0;
+    ksb[u] = 0;
+    if (ci < kKeys * kD / 8) {
+      const int r = ci >> 4, d0 = (ci & 15) * 8;
+      const int32_t slot = row_slot[r];
+      if (slot >= 0) {
+        const int64_t e = ((int64_t)row_token[r] * p.heads + h) * kD + d0;  // element within the slot
+        kcw[u] = *reinterpret_cast<const uint32_t*>(p.base + p.off_k_codes + slot * p.slot_codes_bytes + e / 2);
+        ksb[u] = p.base[p.off_k_scales + slot * p.slot_scales_bytes + e / 16];
+      }
+    }
+  }
+#pragma unroll
+  for (int u = 0; u < kChunksPerThread; ++u) {
+    const int ci = threadIdx.x + u * kThreads;
+    if (ci >= kKeys * kD / 8) break;
     const int r = ci >> 4, c16 = ci & 15;  // key row, 8-value chunk along head_dim
     const int d0 = c16 * 8;
     uint4 out = make_uint4(0, 0, 0, 0);
     const int32_t slot = row_slot[r];
     if (slot >= 0) {
-      const int64_t e = ((int64_t)row_token[r] * p.heads + h) * kD + d0;  // element within the slot
-      const uint32_t kc = *reinterpret_cast<const uint32_t*>(p.base + p.off_k_codes + slot * p.slot_codes_bytes + e / 2);
-      const uint32_t ks2 = e4m3_to_f16x2_bcast(p.base[p.off_k_scales + slot * p.slot_scales_bytes + e / 16]);
+      const uint32_t kc = kcw[u];
+      const uint32_t ks2 = e4m3_to_f16x2_bcast(ksb[u]);
       const float gk = reinterpret_cast<const float*>(p.base + p.off_gscale)[2 * slot];
       const float4* m4 = reinterpret_cast<const float4*>(p.base + p.off_mu + ((int64_t)slot * C + h * kD + d0) * 4);
       const float4 m0 = m4[0], m1 = m4[1];
@@ -255,9 +278,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ epilogue
-    const int quarter = warp & 3;  // the tensor-memory lanes this warp may access
+    // Warp w reads tensor-memory lane quarter w % 4: query rows 32 (w % 4) .. + 31 of
+    // the tile, one per lane.  Each 32-row x 128-byte box of scores (64 bf16 or 32
+    // FP32 keys) is written swizzled into one of the warp's two staging buffers and
+    // stored by TMA, clipped to the head's queries and the window's keys.
+    const int quarter = warp & 3;
     const int64_t key0 = (int64_t)kt * kKeys;
-    const int nkeys = (int)min((int64_t)kKeys, p.Tk - key0);
+    const int cols = p.s_bf16 ? 64 : 32;  // keys per box
+    const uint32_t wbuf = smem_u32(stage) + (uint32_t)((warp - 2) * 2 * kBoxBytes);
+    uint32_t nbox = 0;
     for (uint32_t qt = 0; qt < (uint32_t)n_qt; ++qt) {
       const int a = qt % kAcc;
       if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&t_full[a]), (qt / kAcc) & 1u, abort_flag, limit))) {
@@ -266,50 +295,51 @@ __global__ void __launch_bounds__(kThreads, 1)
         break;
       }
       fence_after();
-      const int64_t qrow = (int64_t)qt * kQ + quarter * 32 + lane;
-      uint8_t* dst = p.s_out + ((int64_t)h * p.head_stride + qrow * p.ld_s + key0) * (p.s_bf16 ? 2 : 4);
+      const uint32_t trow = tmem_base + ((uint32_t)(quarter * 32) << 16) + a * kKeys;
 #pragma unroll 1
-      for (int cc = 0; cc < kKeys; cc += 32) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + a * kKeys + cc, r);
+      for (int c0 = 0; c0 < kKeys && key0 + c0 < p.Tk; c0 += cols, ++nbox) {  // warp-uniform
+        uint32_t w[32];  // the row's 128 bytes of this box
+        {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(trow + c0, r);
+          float v[32];
+#pragma unroll
+          for (int i = 0; i < 32; i += 2)
+            mul2(v[i], v[i + 1], __uint_as_float(r[i]), __uint_as_float(r[i + 1]), p.scale, p.scale);
+          if (p.s_bf16) {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+            tmem_ld_32x32b_x32(trow + c0 + 32, r);
+#pragma unroll
+            for (int i = 0; i < 32; i += 2)
+              mul2(v[i], v[i + 1], __uint_as_float(r[i]), __uint_as_float(r[i + 1]), p.scale, p.scale);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) w[16 + i] = pack_bf16x2(v[2 * i], v[2 * i + 1]);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) w[i] = __float_as_uint(v[i]);
+          }
+        }
+        const uint32_t buf = wbuf + (nbox & 1u) * kBoxBytes;
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
         __syncwarp();
-        if (qrow >= p.Tq || cc >= nkeys) continue;  // no warp-collective work follows in this pass
-        float v[32];
 #pragma unroll
-        for (int i = 0; i < 32; i += 2)
-          mul2(v[i], v[i + 1], __uint_as_float(r[i]), __uint_as_float(r[i + 1]), p.scale, p.scale);
-        const int nv = min(32, nkeys - cc);  // a multiple of 8 unless the window ends here
-        if (p.s_bf16) {
-          uint8_t* d = dst + cc * 2;
-          if (nv == 32) {
-#pragma unroll
-            for (int u = 0; u < 4; ++u)
-              stg_v4(d + 16 * u, make_uint4(pack_bf16x2(v[8 * u], v[8 * u + 1]), pack_bf16x2(v[8 * u + 2], v[8 * u + 3]),
-                                            pack_bf16x2(v[8 * u + 4], v[8 * u + 5]),
-                                            pack_bf16x2(v[8 * u + 6], v[8 * u + 7])));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (i < nv) reinterpret_cast<uint16_t*>(d)[i] = (uint16_t)(pack_bf16x2(v[i], 0.0f) & 0xFFFFu);
-          }
-        } else {
-          float* d = reinterpret_cast<float*>(dst) + cc;
-          if (nv == 32) {
-#pragma unroll
-            for (int u = 0; u < 8; ++u)
-              stg_v4(d + 4 * u, make_uint4(__float_as_uint(v[4 * u]), __float_as_uint(v[4 * u + 1]),
-                                           __float_as_uint(v[4 * u + 2]), __float_as_uint(v[4 * u + 3])));
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if (i < nv) d[i] = v[i];
-          }
+        for (int c = 0; c < 8; ++c)  // 128-byte swizzle: chunk c of row r at chunk c ^ (r % 8)
+          st_shared_v4(buf + lane * 128 + ((c ^ (lane & 7)) << 4),
+                       make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]));
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_3d(&map_s, buf, (int32_t)(key0 + c0), (int32_t)(qt * kQ + quarter * 32), h);
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
         }
       }
       fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&t_empty[a]));
     }
+    if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // stores complete
+    __syncwarp();
   }
 
   fence_before();
@@ -369,10 +399,7 @@ cudaError_t launch_kv_scores(const KVLayout& L, const int32_t* slots, const int3
   p.Tq = tq;
   p.Tk = acc;
   p.scale = scale;
-  p.s_out = static_cast<uint8_t*>(s_out);
   p.s_bf16 = s_bf16;
-  p.ld_s = ld_s;
-  p.head_stride = tq * ld_s;
   p.status = status;
   p.wait_limit_ns = kWaitLimitNs;
   if (tq == 0) return cudaSuccess;
@@ -390,6 +417,19 @@ cudaError_t launch_kv_scores(const KVLayout& L, const int32_t* slots, const int3
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
 
+  // scores [heads][tq][ld_s]: 32-row x 128-byte boxes (64 bf16 or 32 FP32 keys), the
+  // same 128-byte swizzle as the staging buffers; clipped at tq queries and Tk keys
+  CUtensorMap ms;
+  const cuuint64_t esz = s_bf16 ? 2 : 4;
+  cuuint64_t sdims[3] = {(cuuint64_t)acc, (cuuint64_t)tq, (cuuint64_t)L.heads};
+  cuuint64_t sstrides[2] = {(cuuint64_t)ld_s * esz, (cuuint64_t)ld_s * esz * (cuuint64_t)tq};
+  cuuint32_t sbox[3] = {(cuuint32_t)(128 / esz), 32, 1};
+  cuuint32_t sestr[3] = {1, 1, 1};
+  if (fn(&ms, s_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, s_out, sdims,
+         sstrides, sbox, sestr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+
   static std::atomic<bool> done[64];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
@@ -401,7 +441,7 @@ cudaError_t launch_kv_scores(const KVLayout& L, const int32_t* slots, const int3
     done[dev].store(true, std::memory_order_relaxed);
   }
   const dim3 grid((unsigned)((acc + kKeys - 1) / kKeys), (unsigned)L.heads, 1);
-  launch_pdl(kv_scores_kernel, grid, kThreads, kSmemBytes, s, mq, p);
+  launch_pdl(kv_scores_kernel, grid, kThreads, kSmemBytes, s, mq, ms, p);
   return cudaGetLastError();
 }
 

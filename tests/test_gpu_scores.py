@@ -61,12 +61,14 @@ def run_scores(cache, khat, slots, tokens, tq, heads, out_dtype, scale, seed, pa
     return got, ref, bound, tk
 
 
-def assert_scores(got, ref, bound, tk, extra_rel=0.0):
+def assert_scores(got, ref, bound, tk, extra_rel=0.0, esz=4):
     g = got[:, :, :tk]
     err = np.abs(g - ref)
     lim = TOL * bound + extra_rel * np.abs(ref)
     assert np.all(err <= lim), f"{int(np.sum(err > lim))} scores outside the bound"
-    assert np.all(np.isnan(got[:, :, tk:])), "columns beyond the window were written"
+    pad_end = (tk * esz + 15) // 16 * 16 // esz  # the row's next 16-byte boundary
+    assert np.all(got[:, :, tk:pad_end] == 0), "the padding up to the 16-byte boundary holds zeros"
+    assert np.all(np.isnan(got[:, :, pad_end:])), "columns beyond the padding were written"
 
 
 @pytest.mark.parametrize("tq", [1, 128, 200])
@@ -84,7 +86,7 @@ def test_bf16_output_and_repeated_slots(cuda_dev):
     cache, khat = build_cache(heads=3, chunk=192, fills=[192, 192], seed=6)
     slots, tokens = [1, 0, 1], [192, 192, 192]
     got, ref, bound, tk = run_scores(cache, khat, slots, tokens, 300, 3, torch.bfloat16, 0.125, 10)
-    assert_scores(got, ref, bound, tk, extra_rel=2.0 ** -8)
+    assert_scores(got, ref, bound, tk, extra_rel=2.0 ** -8, esz=2)
     assert device_status() == nv.OK
 
 
