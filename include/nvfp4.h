@@ -386,6 +386,19 @@ nvfp4_status nvfp4_get_device_status(int32_t device, int32_t* status_out, int32_
  * Not for use while other GEMM work is in flight. */
 nvfp4_status nvfp4_debug_gemm_fault(int32_t drop_first_stage, uint64_t wait_limit_ns);
 
+/* Test hook for the grid barrier of the one-launch quantization (a tensor that
+ * fits in L2, tensor scale computed from the data), whose CTAs meet inside the
+ * kernel between the amax pass and the encode pass (process-wide; no effect until
+ * called).  Each barrier gives up after a time limit (2 s), records
+ * NVFP4_ERR_TIMEOUT in the device status word and the kernel returns, so the
+ * context stays usable.
+ *   extra_arrivals > 0: every barrier waits for that many CTAs more than the grid
+ *     has, so it runs out: the call ends with device status NVFP4_ERR_TIMEOUT and
+ *     unspecified outputs.  0 restores normal work.
+ *   wait_limit_ns > 0 replaces the 2 s limit; 0 restores it.
+ * Not for use while other work of the library is in flight. */
+nvfp4_status nvfp4_debug_grid_barrier(uint32_t extra_arrivals, uint64_t wait_limit_ns);
+
 /* Human-readable name of a status code (static string). */
 const char* nvfp4_status_string(int32_t status);
 

@@ -69,7 +69,7 @@ EXPORTS = ["nvfp4_version", "nvfp4_status_string", "nvfp4_scales_bytes", "nvfp4_
            "kv_quant_append", "kv_quant_append_noalloc", "kv_dequant_window", "kv_dequant_window_tokens",
            "kv_window_scores",
            "nvfp4_lora_merge", "nvfp4_amax_history_push", "nvfp4_last_cuda_error_string",
-           "nvfp4_debug_gemm_fault",
+           "nvfp4_debug_gemm_fault", "nvfp4_debug_grid_barrier",
            "nvfp4_get_device_status"]
 
 
@@ -88,6 +88,8 @@ def library():
             lib.nvfp4_version.restype = i32
             lib.nvfp4_status_string.restype = ctypes.c_char_p
             lib.nvfp4_status_string.argtypes = [i32]
+            lib.nvfp4_debug_grid_barrier.restype = i32
+            lib.nvfp4_debug_grid_barrier.argtypes = [ctypes.c_uint32, ctypes.c_uint64]
             lib.nvfp4_debug_gemm_fault.restype = i32
             lib.nvfp4_debug_gemm_fault.argtypes = [i32, ctypes.c_uint64]
             lib.nvfp4_last_cuda_error_string.restype = ctypes.c_char_p
@@ -343,6 +345,11 @@ def nvfp4_amax_history_push(history, amax_new, gscale_out, stream=None):
 def debug_gemm_fault(drop_first_stage: bool, wait_limit_ns: int = 0):
     """Test hook of the GEMM's bounded waits (see nvfp4_debug_gemm_fault)."""
     _check(library().nvfp4_debug_gemm_fault(1 if drop_first_stage else 0, wait_limit_ns), "nvfp4_debug_gemm_fault")
+
+
+def debug_grid_barrier(extra_arrivals: int, wait_limit_ns: int = 0):
+    """Test hook of the one-launch quantization's grid barrier (see nvfp4_debug_grid_barrier)."""
+    _check(library().nvfp4_debug_grid_barrier(extra_arrivals, wait_limit_ns), "nvfp4_debug_grid_barrier")
 
 
 def get_device_status(device: int = 0, clear: bool = False) -> int:

@@ -463,6 +463,11 @@ nvfp4_status nvfp4_amax_history_push(float* history, int32_t len, const float* a
                                                 reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_debug_grid_barrier(uint32_t extra_arrivals, uint64_t wait_limit_ns) {
+  nvfp4::grid_barrier_debug(extra_arrivals, (unsigned long long)wait_limit_ns);
+  return NVFP4_OK;
+}
+
 nvfp4_status nvfp4_debug_gemm_fault(int32_t drop_first_stage, uint64_t wait_limit_ns) {
   nvfp4::gemm_debug_fault(drop_first_stage, (unsigned long long)wait_limit_ns);
   return NVFP4_OK;

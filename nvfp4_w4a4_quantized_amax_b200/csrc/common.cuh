@@ -119,10 +119,10 @@ constexpr unsigned long long kGridBarrierLimitNs = 2000000000ull;
 // Barrier of a whole grid whose CTAs are all resident at once (one wave, sized by
 // the occupancy query, launched after every earlier grid on the stream has
 // started).  *ctr is zero before the launch; each CTA adds one and waits for
-// gridDim.x arrivals.  The wait is bounded: false after limit_ns, and the caller
+// `expected` arrivals (every CTA of the grid).  The wait is bounded: false after limit_ns, and the caller
 // records a timeout instead of hanging.  Memory written by any CTA before the
 // barrier is visible to every CTA after it (release/acquire at GPU scope).
-__device__ __forceinline__ bool grid_barrier(unsigned* ctr, unsigned long long limit_ns) {
+__device__ __forceinline__ bool grid_barrier_n(unsigned* ctr, unsigned expected, unsigned long long limit_ns) {
   __shared__ int barrier_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
@@ -130,7 +130,7 @@ __device__ __forceinline__ bool grid_barrier(unsigned* ctr, unsigned long long l
     atomicAdd(ctr, 1u);
     int ok = 1;
     const unsigned long long t0 = globaltimer_ns();
-    while (ld_acquire_gpu(ctr) < gridDim.x) {
+    while (ld_acquire_gpu(ctr) < expected) {
       if (globaltimer_ns() - t0 > limit_ns) {
         ok = 0;
         break;

@@ -118,6 +118,13 @@ cudaError_t launch_kv_scores(const KVLayout& c, const int32_t* slots, const int3
                              const void* q, int64_t tq, int64_t ldq, float scale, void* s_out, bool s_bf16,
                              int64_t ld_s, unsigned* status, cudaStream_t s);
 
+// Test hook of the grid barrier of the one-launch quantization (see
+// nvfp4_debug_grid_barrier): arrivals a barrier waits for beyond the grid's CTAs
+// (0 = none) and its time limit (0 = the default 2 s).
+void grid_barrier_debug(unsigned extra, unsigned long long limit_ns);
+unsigned grid_barrier_extra();
+unsigned long long grid_barrier_limit_ns();
+
 // Zero n_words 32-bit words of device memory (a PDL-launched kernel, not a memset).
 cudaError_t launch_zero_words(void* p, int n_words, cudaStream_t s);
 

@@ -200,7 +200,9 @@ __device__ unsigned g_grid_sync[kGridSyncSlots];
 // met, so a dependent grid can never hold resources that one of its CTAs still needs.
 template <bool kBf16, bool kMma>
 __global__ void __launch_bounds__(kThreads) quantize_fused_kernel(EncodeParams p, unsigned* amax_bits,
-                                                                  int slot, int64_t nchunks, FastDiv cpr) {
+                                                                  int slot, int64_t nchunks, FastDiv cpr,
+                                                                  unsigned barrier_extra,
+                                                                  unsigned long long barrier_limit_ns) {
   pdl_wait();
   const int64_t stride = (int64_t)gridDim.x * kThreads;
   const int64_t first = (int64_t)blockIdx.x * kThreads + threadIdx.x;
@@ -225,7 +227,7 @@ __global__ void __launch_bounds__(kThreads) quantize_fused_kernel(EncodeParams p
   }
   if (kBf16) m = max(m >> 16, m & 0xFFFFu) << 16;
   block_max_atomic(m, amax_bits);
-  if (!grid_barrier(&g_grid_sync[slot], kGridBarrierLimitNs)) {
+  if (!grid_barrier_n(&g_grid_sync[slot], gridDim.x + barrier_extra, barrier_limit_ns)) {
     if (threadIdx.x == 0) set_status(p.status, kStatusTimeout);
     pdl_trigger();
     return;
@@ -384,7 +386,7 @@ static cudaError_t launch_fused(const EncodeParams& p, unsigned* amax_bits, cuda
   const int grid = wave_grid<quantize_fused_kernel<kBf16, kMma>>(kThreads, p.nvblocks);
   const int64_t cpr = p.nb * (kBf16 ? 2 : 4);  // 16-byte chunks of x per row
   launch_pdl(quantize_fused_kernel<kBf16, kMma>, grid, kThreads, 0, s, p, amax_bits, slot, p.rows * cpr,
-             FastDiv((uint32_t)cpr));
+             FastDiv((uint32_t)cpr), grid_barrier_extra(), grid_barrier_limit_ns());
   return cudaGetLastError();
 }
 
@@ -469,6 +471,21 @@ cudaError_t launch_dequantize(const DequantizeArgs& a, cudaStream_t s) {
 }  // namespace nvfp4
 
 namespace nvfp4 {
+namespace {
+std::atomic<unsigned> g_barrier_extra{0};
+std::atomic<unsigned long long> g_barrier_limit_ns{0};
+}  // namespace
+
+void grid_barrier_debug(unsigned extra, unsigned long long limit_ns) {
+  g_barrier_extra.store(extra);
+  g_barrier_limit_ns.store(limit_ns);
+}
+unsigned grid_barrier_extra() { return g_barrier_extra.load(); }
+unsigned long long grid_barrier_limit_ns() {
+  const unsigned long long v = g_barrier_limit_ns.load();
+  return v ? v : kGridBarrierLimitNs;
+}
+
 cudaError_t launch_zero_words(void* p, int n_words, cudaStream_t s) {
   launch_pdl(zero_words_kernel, 1, 32, 0, s, static_cast<unsigned*>(p), n_words);
   return cudaGetLastError();

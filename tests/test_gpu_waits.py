@@ -1,7 +1,8 @@
-"""Bounded waits of the GEMM kernels: with the test hook that makes every CTA's
-producer skip its first pipeline stage, the waits for that stage run out, the
-call reports NVFP4_ERR_TIMEOUT in the device status word, returns in bounded time,
-and the context stays usable (the next GEMM is correct)."""
+"""Bounded waits: with the test hook that makes every CTA's GEMM producer skip its
+first pipeline stage, or the one that makes the grid barrier of the one-launch
+quantize wait for more CTAs than the grid has, the waits run out,
+the call reports NVFP4_ERR_TIMEOUT in the device status word, returns in bounded
+time, and the context stays usable (the next call is correct)."""
 import time
 
 import numpy as np
@@ -11,7 +12,7 @@ import torch
 import nvfp4_w4a4_quantized_amax_b200 as nv
 import oracle
 import synth
-from gpu_helpers import canonical, device_status, gpu_quantize
+from gpu_helpers import assert_quant_equal, canonical, dev_bf16, device_status, gpu_quantize
 
 pytestmark = pytest.mark.gpu
 
@@ -40,3 +41,20 @@ def test_gemm_wait_timeout_is_reported_and_the_context_survives(cuda_dev, M, N, 
     wc, wsc, wg = canonical(qw)
     ref, bound = oracle.gemm_ref(ac, asc, ag, wc, wsc, wg)
     assert np.all(np.abs(c.cpu().numpy().astype(np.float64) - ref) <= 1e-5 * bound)
+
+
+def test_grid_barrier_timeout_in_one_launch_quantize(cuda_dev):
+    x = synth.activations(42, 512, 1024)  # small: the one-launch path
+    assert device_status(clear=True) == nv.OK
+    nv.debug_grid_barrier(1, 20_000_000)  # one CTA more than the grid has, 20 ms
+    try:
+        t0 = time.time()
+        gpu_quantize(x, nv.SF_MMA)
+        elapsed = time.time() - t0
+    finally:
+        nv.debug_grid_barrier(0, 0)
+    assert device_status(clear=True) == nv.ERR_TIMEOUT
+    assert elapsed < 5.0
+    q, _ = gpu_quantize(x, nv.SF_MMA)
+    assert device_status() == nv.OK
+    assert_quant_equal(q, oracle.quantize(x))
