@@ -333,6 +333,27 @@ nvfp4_status kv_window_scores(const nvfp4_kv_cache* cache, const int32_t* slots_
                               int32_t n_slots, const void* q, int64_t tq, int64_t ldq, float scale, void* s_out,
                               int32_t st, int64_t ld_s, nvfp4_stream_t stream);
 
+/* kv_window_context — the V side of attention from the NVFP4 cache: the weighted
+ * sum of the window's values, O = P V^, with V dequantized inside the kernel (one
+ * 128-key tile at a time, into shared memory; no bf16 copy of the window's V is
+ * written).  [TW] §四, as for kv_window_scores.
+ *   slots_host, tokens_host, n_slots : the window (HOST arrays), Tk keys in list
+ *              order, exactly as for kv_dequant_window_tokens.
+ *   p        : device bf16 [heads][tq][ld_p] weights of the keys (e.g. the softmax
+ *              of kv_window_scores' output), ld_p >= Tk; base and row pitch 16-byte
+ *              aligned.  Elements beyond Tk in a row are not read.
+ *   o_out    : device [tq][heads][head_dim] of ot (NVFP4_FP32 or NVFP4_BF16), row
+ *              pitch ldo elements (>= heads * head_dim), base and pitch 16-byte aligned:
+ *                O[i, h, d] = sum_j p[h, i, j] * V^[j, h, d],
+ *              accumulated in FP32 by the tensor cores, V^ bit for bit the window's V
+ *              that kv_dequant_window_tokens writes; bf16 output is the RNE of it.
+ * Requires head_dim == 128.  A listed slot whose recorded token count differs sets
+ * device status NVFP4_ERR_SHAPE (its keys then count as zero).  Errors:
+ * INVALID_ARG, SHAPE, ALIGNMENT. */
+nvfp4_status kv_window_context(const nvfp4_kv_cache* cache, const int32_t* slots_host, const int32_t* tokens_host,
+                               int32_t n_slots, const void* p, int64_t tq, int64_t ld_p, void* o_out, int32_t ot,
+                               int64_t ldo, nvfp4_stream_t stream);
+
 /* ----------------------------------------------------------- amax history ----
  * A requantizing GEMM epilogue (nvfp4_epilogue.q_out) quantizes before its own
  * max|h| is known, so it takes a supplied tensor scale (q_gscale_in) and reports

@@ -67,7 +67,7 @@ class nvfp4_kv_cache(ctypes.Structure):
 EXPORTS = ["nvfp4_version", "nvfp4_status_string", "nvfp4_scales_bytes", "nvfp4_quantize", "nvfp4_amax",
            "nvfp4_dequantize", "nvfp4_gemm", "nvfp4_kv_cache_bytes", "nvfp4_kv_cache_init",
            "kv_quant_append", "kv_quant_append_noalloc", "kv_dequant_window", "kv_dequant_window_tokens",
-           "kv_window_scores",
+           "kv_window_scores", "kv_window_context",
            "nvfp4_lora_merge", "nvfp4_amax_history_push", "nvfp4_last_cuda_error_string",
            "nvfp4_debug_gemm_fault", "nvfp4_debug_grid_barrier",
            "nvfp4_get_device_status"]
@@ -120,6 +120,9 @@ def library():
             lib.kv_window_scores.restype = i32
             lib.kv_window_scores.argtypes = [KV, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), i32,
                                              vp, i64, i64, ctypes.c_float, vp, i32, i64, vp]
+            lib.kv_window_context.restype = i32
+            lib.kv_window_context.argtypes = [KV, ctypes.POINTER(ctypes.c_int32), ctypes.POINTER(ctypes.c_int32), i32,
+                                              vp, i64, i64, vp, i32, i64, vp]
             lib.nvfp4_lora_merge.restype = i32
             lib.nvfp4_lora_merge.argtypes = [vp, i32, i64, i64, i64, vp, vp, i32, ctypes.c_float, vp, i64, vp]
             lib.nvfp4_amax_history_push.restype = i32
@@ -322,6 +325,18 @@ def kv_window_scores(cache: KVCache, slots: Sequence[int], tokens: Sequence[int]
     _check(library().kv_window_scores(ctypes.byref(cache.handle), sarr, tarr, len(slots), _ptr(q), tq,
                                       q.stride(0), float(scale), _ptr(s_out), _dtype_code(s_out),
                                       s_out.stride(1), _stream(stream)), "kv_window_scores")
+
+
+def kv_window_context(cache: KVCache, slots: Sequence[int], tokens: Sequence[int], p, o_out, stream=None):
+    """O = P V^ over the window's keys, V read from the NVFP4 cache inside the kernel:
+    p bf16 [heads, tq, >= Tk]; o_out (fp32 or bf16) [tq, heads, head_dim]."""
+    if len(tokens) != len(slots):
+        raise ValueError("one token count per slot")
+    sarr = (ctypes.c_int32 * len(slots))(*slots)
+    tarr = (ctypes.c_int32 * len(tokens))(*tokens)
+    _check(library().kv_window_context(ctypes.byref(cache.handle), sarr, tarr, len(slots), _ptr(p), p.shape[1],
+                                       p.stride(1), _ptr(o_out), _dtype_code(o_out), o_out.stride(0),
+                                       _stream(stream)), "kv_window_context")
 
 
 def nvfp4_lora_merge(w, lora_b, lora_a, scale: float, out, stream=None):

@@ -416,6 +416,32 @@ nvfp4_status kv_window_scores(const nvfp4_kv_cache* cache, const int32_t* slots_
                                              reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status kv_window_context(const nvfp4_kv_cache* cache, const int32_t* slots_host, const int32_t* tokens_host,
+                               int32_t n_slots, const void* p, int64_t tq, int64_t ld_p, void* o_out, int32_t ot,
+                               int64_t ldo, nvfp4_stream_t stream) {
+  nvfp4::KVLayout L;
+  nvfp4_status st_ = check_cache(cache, &L, /*needs_scratch=*/false);
+  if (st_ != NVFP4_OK) return st_;
+  if (!slots_host || !tokens_host || !o_out || (!p && tq > 0) || !valid_dtype(ot)) return NVFP4_ERR_INVALID_ARG;
+  if (n_slots < 1 || n_slots > nvfp4::kMaxWindowSlots) return NVFP4_ERR_INVALID_ARG;
+  if (cache->head_dim != 128) return NVFP4_ERR_SHAPE;
+  int64_t total = 0;
+  for (int i = 0; i < n_slots; ++i) {
+    if (slots_host[i] < 0 || slots_host[i] >= cache->max_chunks) return NVFP4_ERR_INVALID_ARG;
+    if (tokens_host[i] < 1 || tokens_host[i] > cache->chunk_tokens) return NVFP4_ERR_SHAPE;
+    total += tokens_host[i];
+  }
+  const int64_t esz = ot == NVFP4_BF16 ? 2 : 4;
+  if (tq < 0 || ld_p < total || ldo < (int64_t)cache->heads * 128) return NVFP4_ERR_SHAPE;
+  if (tq > (1ll << 31) || total > (1ll << 31) || (int64_t)cache->heads > 65535) return NVFP4_ERR_SHAPE;
+  if (tq > 0 && (!aligned16(p) || (ld_p * 2) % 16 != 0)) return NVFP4_ERR_ALIGNMENT;
+  if (!aligned16(o_out) || (ldo * esz) % 16 != 0) return NVFP4_ERR_ALIGNMENT;
+  unsigned* status = nullptr;
+  if ((st_ = current_device(&status)) != NVFP4_OK) return st_;
+  return cuda_status(nvfp4::launch_kv_context(L, slots_host, tokens_host, n_slots, p, tq, ld_p, o_out,
+                                              ot == NVFP4_BF16, ldo, status, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status kv_dequant_window(const nvfp4_kv_cache* cache, const int32_t* slots_host,
                                int32_t n_slots, void* k_out, void* v_out, nvfp4_stream_t stream) {
   if (!cache || n_slots < 1 || n_slots > nvfp4::kMaxWindowSlots) return NVFP4_ERR_INVALID_ARG;

@@ -118,6 +118,12 @@ cudaError_t launch_kv_scores(const KVLayout& c, const int32_t* slots, const int3
                              const void* q, int64_t tq, int64_t ldq, float scale, void* s_out, bool s_bf16,
                              int64_t ld_s, unsigned* status, cudaStream_t s);
 
+// Attention output O [tq][heads][128] (row pitch ldo) = P V^ over the window's keys,
+// P bf16 [heads][tq][ld_p], V dequantized from the cache inside the kernel.
+cudaError_t launch_kv_context(const KVLayout& c, const int32_t* slots, const int32_t* tokens, int32_t n_slots,
+                              const void* p, int64_t tq, int64_t ld_p, void* o_out, bool o_bf16, int64_t ldo,
+                              unsigned* status, cudaStream_t s);
+
 // Test hook of the grid barrier of the one-launch quantization (see
 // nvfp4_debug_grid_barrier): arrivals a barrier waits for beyond the grid's CTAs
 // (0 = none) and its time limit (0 = the default 2 s).

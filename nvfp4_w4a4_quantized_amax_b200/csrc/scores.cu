@@ -352,6 +352,284 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ============================================================ the V side
+// O[i, h, d] = sum_j P[h, i, j] * V^[j, h, d] over the window's keys j, with
+//   V^[j, h, d] = bf16(RN(RN(e2m1 * s) * g_V))   (the window's V, bit for bit)
+// and P given (e.g. the softmax of the scores), FP32 accumulation in tensor memory.
+// CTA (128-query tile, head), 8 warps:
+//   warp 0      TMA producer: P tiles (128 queries x 128 keys bf16, two 64-key boxes,
+//               128-byte swizzle), double-buffered
+//   warp 1      MMA issuer: 8 tcgen05.mma (K = 16 keys each) per key tile into one
+//               128 x 128 FP32 accumulator
+//   warps 4..7  dequantize each key tile's V^ from the cache straight into shared
+//               memory, transposed (128 dims x 128 keys, K-major for the MMA's B
+//               operand), double-buffered; at the end the epilogue (one lane
+//               quarter each): the 128 outputs of a query row, staged in shared
+//               memory and written by TMA stores clipped to the query count.
+constexpr int kCtxThreads = 256;
+constexpr int kCtxBufs = 2;
+constexpr int kPBytes = kQ * kKeys * 2;  // 32 KB
+constexpr int kVBytes = kD * kKeys * 2;  // 32 KB
+constexpr int kCtxSmemBytes = kCtxBufs * (kPBytes + kVBytes) + 1024 /*barriers*/ + 1024 /*alignment*/;
+constexpr int kCtxTmemCols = kD;         // one 128-column accumulator
+constexpr int kVWarp0 = 4;
+
+struct ContextParams {
+  const uint8_t* base;
+  int64_t off_v_codes, off_v_scales, off_gscale, off_tokens;
+  int64_t slot_codes_bytes, slot_scales_bytes;
+  int32_t heads, n_slots;
+  int32_t slots[kMaxWindowSlots];
+  int32_t tokens[kMaxWindowSlots];
+  int64_t key_end[kMaxWindowSlots];
+  int64_t Tq, Tk;
+  bool o_bf16;
+  unsigned* status;
+  unsigned long long wait_limit_ns;
+};
+
+// kind::f16 again (M = N = 128); the B operand is V^ transposed (dims x keys).
+__global__ void __launch_bounds__(kCtxThreads, 1)
+    kv_context_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ CUtensorMap map_o,
+                      ContextParams p) {
+  pdl_trigger();
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* pbuf = smem;                                // kCtxBufs P tiles
+  uint8_t* vbuf = smem + kCtxBufs * kPBytes;           // kCtxBufs V^T tiles
+  uint8_t* bar_area = vbuf + kCtxBufs * kVBytes;
+  uint64_t* p_full = reinterpret_cast<uint64_t*>(bar_area);
+  uint64_t* p_empty = p_full + kCtxBufs;
+  uint64_t* v_full = p_empty + kCtxBufs;
+  uint64_t* v_empty = v_full + kCtxBufs;
+  uint64_t* t_full = v_empty + kCtxBufs;
+  uint64_t* done_bar = t_full + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qt = blockIdx.x, h = blockIdx.y;
+  const int64_t n_kt = (p.Tk + kKeys - 1) / kKeys;
+  const unsigned long long limit = p.wait_limit_ns;
+
+  if (threadIdx.x == 0) {
+    for (int b = 0; b < kCtxBufs; ++b) {
+      mbar_init(smem_u32(&p_full[b]), 1);
+      mbar_init(smem_u32(&p_empty[b]), 1);
+      mbar_init(smem_u32(&v_full[b]), 4);
+      mbar_init(smem_u32(&v_empty[b]), 1);
+    }
+    mbar_init(smem_u32(t_full), 1);
+    mbar_init(smem_u32(done_bar), 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  if (warp == 0) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tmem_slot)),
+                 "r"(kCtxTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  fence_before();
+  __syncthreads();
+  fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // the cache and P come from earlier work
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ P producer
+    if (lane == 0) {
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_p)) : "memory");
+      bool ok = true;
+      uint32_t issued = 0;
+      for (uint32_t kt = 0; kt < (uint32_t)n_kt; ++kt) {
+        const int b = kt % kCtxBufs;
+        if (!mbar_wait(smem_u32(&p_empty[b]), ((kt / kCtxBufs) & 1u) ^ 1u, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        const uint32_t fb = smem_u32(&p_full[b]);
+        mbar_arrive_expect_tx(fb, kPBytes);
+        uint8_t* dst = pbuf + b * kPBytes;
+        tma_load_3d(smem_u32(dst), &map_p, fb, (int32_t)(kt * kKeys), qt * kQ, h);
+        tma_load_3d(smem_u32(dst + kBlockBytes), &map_p, fb, (int32_t)(kt * kKeys + 64), qt * kQ, h);
+        issued = kt + 1;
+      }
+      if (!ok) {
+        set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+      for (uint32_t j = issued > (uint32_t)kCtxBufs ? issued - kCtxBufs : 0; j < issued; ++j)
+        mbar_wait_drain(smem_u32(&p_full[j % kCtxBufs]), (j / kCtxBufs) & 1u, limit);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      bool ok = true;
+      for (uint32_t kt = 0; kt < (uint32_t)n_kt; ++kt) {
+        const int b = kt % kCtxBufs;
+        const uint32_t ph = (kt / kCtxBufs) & 1u;
+        if (!mbar_wait(smem_u32(&v_full[b]), ph, abort_flag, limit) ||
+            !mbar_wait(smem_u32(&p_full[b]), ph, abort_flag, limit)) {
+          ok = false;
+          break;
+        }
+        fence_after();
+        const uint32_t a_addr = smem_u32(pbuf + b * kPBytes), b_addr = smem_u32(vbuf + b * kVBytes);
+#pragma unroll
+        for (int kk = 0; kk < kKeys / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
+          mma_bf16(tmem_base, smem_desc(a_addr + off, 16, 1024, 2), smem_desc(b_addr + off, 16, 1024, 2),
+                   (kt > 0 || kk > 0) ? 1u : 0u);
+        }
+        commit(smem_u32(&p_empty[b]));
+        commit(smem_u32(&v_empty[b]));
+      }
+      if (!ok) {
+        set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+      } else {
+        commit(smem_u32(t_full));
+      }
+      commit(smem_u32(done_bar));
+      mbar_wait_drain(smem_u32(done_bar), 0, limit);
+    }
+  } else if (warp >= kVWarp0) {
+    // ------------------------------------------------------------ V^T producers, then epilogue
+    const int t = threadIdx.x - kVWarp0 * 32;  // 0..127
+    const int kp = t & 63;                     // key pair of the tile: keys 2 kp, 2 kp + 1
+    const int dh = t >> 6;                     // dims [64 dh, 64 dh + 64)
+    bool ok = true;
+    for (uint32_t kt = 0; kt < (uint32_t)n_kt && ok; ++kt) {
+      const int b = kt % kCtxBufs;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&v_empty[b]), ((kt / kCtxBufs) & 1u) ^ 1u, abort_flag,
+                                             limit))) {
+        ok = false;
+        break;
+      }
+      fence_after();
+      // the 64 dims of each of the two keys, decoded to bf16 (zeros beyond the window)
+      uint32_t vals[2][32];  // [key][dim pair] as bf16x2 along dims
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int64_t j = (int64_t)kt * kKeys + 2 * kp + e;
+        int32_t slot = -1;
+        int64_t tok = 0;
+        if (j < p.Tk) {
+          int i = 0;
+          while (j >= p.key_end[i]) ++i;
+          const int64_t begin = i == 0 ? 0 : p.key_end[i - 1];
+          if (reinterpret_cast<const int32_t*>(p.base + p.off_tokens)[p.slots[i]] == p.tokens[i]) {
+            slot = p.slots[i];
+            tok = j - begin;
+          } else if (j == begin) {
+            set_status(p.status, kStatusShape);  // the slot holds another token count
+          }
+        }
+#pragma unroll
+        for (int q = 0; q < 32; ++q) vals[e][q] = 0;
+        if (slot >= 0) {
+          const int64_t el = (tok * p.heads + h) * kD + dh * 64;  // element within the slot
+          const uint8_t* cp = p.base + p.off_v_codes + slot * p.slot_codes_bytes + el / 2;
+          const uint4 c0 = *reinterpret_cast<const uint4*>(cp), c1 = *reinterpret_cast<const uint4*>(cp + 16);
+          const uint32_t sc4 = *reinterpret_cast<const uint32_t*>(p.base + p.off_v_scales + slot * p.slot_scales_bytes + el / 16);
+          const float gv = reinterpret_cast<const float*>(p.base + p.off_gscale)[2 * slot + 1];
+          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+#pragma unroll
+          for (int g8 = 0; g8 < 8; ++g8) {  // 8 dims per code word, 16 per scale byte
+            uint32_t hv[4];
+            e2m1x8_times_scale(cw[g8], e4m3_to_f16x2_bcast((sc4 >> (8 * (g8 >> 1))) & 0xFFu), hv);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              float lo, hi;
+              f16x2_to_f32x2(hv[q], lo, hi);  // e2m1 * s, exact
+              vals[e][g8 * 4 + q] = pack_bf16x2(lo * gv, hi * gv);
+            }
+          }
+        }
+      }
+      // transposed store: row d holds keys along the row; one 32-bit store carries keys
+      // 2 kp and 2 kp + 1 of dim d (128-byte swizzle on 16-byte chunks)
+      uint8_t* vb = vbuf + b * kVBytes;
+      const int col = 2 * kp;                 // key within the tile (even)
+      const int blk = col >> 6, cb = col & 63;
+#pragma unroll
+      for (int q = 0; q < 32; ++q) {
+#pragma unroll
+        for (int e2 = 0; e2 < 2; ++e2) {      // dims 2 q and 2 q + 1 of this half
+          const int d = dh * 64 + 2 * q + e2;
+          const uint32_t lo = e2 ? (vals[0][q] >> 16) : (vals[0][q] & 0xFFFFu);
+          const uint32_t hi = e2 ? (vals[1][q] >> 16) : (vals[1][q] & 0xFFFFu);
+          *reinterpret_cast<uint32_t*>(vb + blk * kBlockBytes + d * 128 + ((((cb >> 3) ^ (d & 7))) << 4) +
+                                       (cb & 7) * 2) = lo | (hi << 16);
+        }
+      }
+      fence_proxy_async_smem();  // the tensor core reads V^T through the async proxy
+      __syncwarp();
+      if (lane == 0) mbar_arrive(smem_u32(&v_full[b]));
+    }
+    if (!ok) {
+      if (lane == 0) set_status(p.status, kStatusTimeout);
+      *abort_flag = 1;
+    } else {
+      // epilogue: warp w reads tensor-memory lane quarter w % 4 (query rows 32 (w % 4) ..)
+      const int quarter = warp & 3;
+      if (__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(t_full), 0, abort_flag, limit))) {
+        fence_after();
+        // the P buffers are free once every MMA has completed: 8 KB of staging per warp
+        const uint32_t wbuf = smem_u32(pbuf) + (uint32_t)((warp - kVWarp0) * 2 * kBoxBytes);
+        const int cols = p.o_bf16 ? 64 : 32;
+        uint32_t nbox = 0;
+        for (int c0 = 0; c0 < kD; c0 += cols, ++nbox) {
+          uint32_t w[32];
+          {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + c0, r);
+            if (p.o_bf16) {
+#pragma unroll
+              for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+              tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + c0 + 32, r);
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                w[16 + i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            } else {
+#pragma unroll
+              for (int i = 0; i < 32; ++i) w[i] = r[i];
+            }
+          }
+          const uint32_t buf = wbuf + (nbox & 1u) * kBoxBytes;
+          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            st_shared_v4(buf + lane * 128 + ((c ^ (lane & 7)) << 4),
+                         make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]));
+          fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&map_o, buf, h * kD + c0, qt * kQ + quarter * 32);
+            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+          }
+        }
+        if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+        __syncwarp();
+      } else {
+        if (lane == 0) set_status(p.status, kStatusTimeout);
+        *abort_flag = 1;
+      }
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+  if (warp == 0) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kCtxTmemCols)
+                 : "memory");
+  }
+}
+
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -442,6 +720,76 @@ cudaError_t launch_kv_scores(const KVLayout& L, const int32_t* slots, const int3
   }
   const dim3 grid((unsigned)((acc + kKeys - 1) / kKeys), (unsigned)L.heads, 1);
   launch_pdl(kv_scores_kernel, grid, kThreads, kSmemBytes, s, mq, ms, p);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4
+
+namespace nvfp4 {
+
+cudaError_t launch_kv_context(const KVLayout& L, const int32_t* slots, const int32_t* tokens, int32_t n_slots,
+                              const void* pm, int64_t tq, int64_t ld_p, void* o_out, bool o_bf16, int64_t ldo,
+                              unsigned* status, cudaStream_t s) {
+  if (L.head_dim != kD) return cudaErrorInvalidValue;
+  ContextParams p;
+  memset(&p, 0, sizeof(p));
+  p.base = L.base;
+  p.off_v_codes = L.off_v_codes;
+  p.off_v_scales = L.off_v_scales;
+  p.off_gscale = L.off_gscale;
+  p.off_tokens = L.off_tokens;
+  p.slot_codes_bytes = L.slot_codes_bytes;
+  p.slot_scales_bytes = L.slot_scales_bytes;
+  p.heads = L.heads;
+  p.n_slots = n_slots;
+  int64_t acc = 0;
+  for (int i = 0; i < n_slots; ++i) {
+    p.slots[i] = slots[i];
+    p.tokens[i] = tokens[i];
+    acc += tokens[i];
+    p.key_end[i] = acc;
+  }
+  p.Tq = tq;
+  p.Tk = acc;
+  p.o_bf16 = o_bf16;
+  p.status = status;
+  p.wait_limit_ns = kWaitLimitNs;
+  if (tq == 0) return cudaSuccess;
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return cudaErrorInvalidValue;
+  // P [heads][tq][ld_p] bf16: 64-key x 128-query boxes, 128-byte swizzle, zero-filled
+  // beyond the window's keys and the query count
+  CUtensorMap mp;
+  cuuint64_t pdims[3] = {(cuuint64_t)acc, (cuuint64_t)tq, (cuuint64_t)L.heads};
+  cuuint64_t pstrides[2] = {(cuuint64_t)ld_p * 2, (cuuint64_t)ld_p * 2 * (cuuint64_t)tq};
+  cuuint32_t pbox[3] = {64, (cuuint32_t)kQ, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  if (fn(&mp, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(pm), pdims, pstrides, pbox, estr,
+         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  // O [tq][heads * 128] (row pitch ldo): 32-row x 128-byte boxes, clipped at tq rows
+  CUtensorMap mo;
+  const cuuint64_t esz = o_bf16 ? 2 : 4;
+  cuuint64_t odims[2] = {(cuuint64_t)L.heads * kD, (cuuint64_t)tq};
+  cuuint64_t ostrides[1] = {(cuuint64_t)ldo * esz};
+  cuuint32_t obox[2] = {(cuuint32_t)(128 / esz), 32};
+  if (fn(&mo, o_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, o_out, odims,
+         ostrides, obox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    return cudaErrorInvalidValue;
+  static std::atomic<bool> done[64];
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  if (!done[dev].load(std::memory_order_relaxed)) {
+    e = cudaFuncSetAttribute(kv_context_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCtxSmemBytes);
+    if (e != cudaSuccess) return e;
+    done[dev].store(true, std::memory_order_relaxed);
+  }
+  const dim3 grid((unsigned)((tq + kQ - 1) / kQ), (unsigned)L.heads, 1);
+  launch_pdl(kv_context_kernel, grid, kCtxThreads, kCtxSmemBytes, s, mp, mo, p);
   return cudaGetLastError();
 }
 

@@ -1,8 +1,10 @@
-"""GPU parity of kv_window_scores (attention scores with K read from the NVFP4 cache
-inside the kernel) against the oracle: the float64 product of the queries with the
-oracle's dequantized K of the window (techwalker.com, "NVIDIA研究团队打造全球首个FP4视频
-生成系统，速度提升两倍还省一半内存", §四: the window's cache chunks are dequantized
-together for attention).  Every score within 1e-5 of sum_d |q_d k_d| (times |scale|)
+"""GPU parity of the attention-side consumers of the NVFP4 KV cache against the
+oracle (techwalker.com, "NVIDIA研究团队打造全球首个FP4视频生成系统，速度提升两倍还省一半内存",
+§四: the window's cache chunks are dequantized together for attention):
+kv_window_scores (K read from the cache inside the kernel) against the float64
+product of the queries with the oracle's dequantized K, and kv_window_context (V read
+from the cache inside the kernel) against the float64 product of the weights with the
+oracle's dequantized V.  Every output within 1e-5 of the sum of the absolute products
 of the exact value; bf16 outputs add half a bf16 ulp."""
 import numpy as np
 import pytest
@@ -18,19 +20,21 @@ pytestmark = pytest.mark.gpu
 TOL = 1e-5
 
 
-def build_cache(heads, chunk, fills, seed):
-    """A cache whose slot s holds fills[s] tokens; the oracle's K^ of each slot."""
+def build_cache(heads, chunk, fills, seed, with_v=False):
+    """A cache whose slot s holds fills[s] tokens; the oracle's K^ (and V^) of each slot."""
     D = 128
     off = synth.kv_offsets(seed, heads, D)
     cache = nv.KVCache(heads, D, chunk, len(fills))
-    khat = []
+    khat, vhat = [], []
     for s, n in enumerate(fills):
         k, v = synth.kv_chunk(seed, s, chunk, heads, D, off)
         k, v = k[:n].copy(), v[:n].copy()
         nv.kv_quant_append(cache, dev_bf16(k), dev_bf16(v), s)
-        khat.append(oracle.kv_dequant_chunk(oracle.kv_append(k, v))[0])
+        kh, vh = oracle.kv_dequant_chunk(oracle.kv_append(k, v))
+        khat.append(kh)
+        vhat.append(vh)
     torch.cuda.synchronize()
-    return cache, khat
+    return (cache, khat, vhat) if with_v else (cache, khat)
 
 
 def reference(q_bits, khat, slots, tokens, scale):
@@ -148,3 +152,100 @@ def test_full_size_window_sampled_heads(cuda_dev):
         bound = (np.abs(qf) @ np.abs(kf).T) / np.sqrt(128.0)
         got = s_out[h].cpu().numpy().astype(np.float64)
         assert np.all(np.abs(got - ref) <= TOL * bound), f"head {h}"
+
+
+# ------------------------------------------------------------------ the V side
+
+def weights(seed, heads, tq, ld):
+    """bf16 weights in [0, 1) with a ragged row pitch beyond the window (NaN there:
+    the kernel must not read past Tk)."""
+    rng = np.random.default_rng(seed)
+    w = rng.random((heads, tq, ld)).astype(np.float32)
+    bits = (w.view(np.uint32) >> 16).astype(np.uint16)
+    return bits
+
+
+def run_context(cache, vhat, slots, tokens, tq, heads, out_dtype, seed):
+    tk = int(sum(tokens))
+    ld = (tk + 16 + 7) // 8 * 8
+    pb = weights(seed, heads, tq, ld)
+    pb[:, :, tk:] = 0x7FC0  # NaN beyond the window
+    o = torch.full((tq, heads, 128), float("nan"), dtype=out_dtype, device="cuda")
+    nv.kv_window_context(cache, slots, tokens, dev_bf16(pb), o)
+    torch.cuda.synchronize()
+    vals = np.concatenate([vhat[s][:t] for s, t in zip(slots, tokens)])     # [Tk, H, D]
+    pf = synth.bf16_bits_to_f32(pb[:, :, :tk]).astype(np.float64)            # [H, Tq, Tk]
+    vf = synth.bf16_bits_to_f32(vals).astype(np.float64)
+    ref = np.einsum("hij,jhd->ihd", pf, vf)
+    bound = np.einsum("hij,jhd->ihd", np.abs(pf), np.abs(vf))
+    return o.float().cpu().numpy().astype(np.float64), ref, bound
+
+
+@pytest.mark.parametrize("tq", [1, 130])
+def test_context_ragged_window(cuda_dev, tq):
+    cache, _, vhat = build_cache(heads=2, chunk=256, fills=[256, 200, 77], seed=15, with_v=True)
+    got, ref, bound = run_context(cache, vhat, [2, 0, 1], [77, 256, 200], tq, 2, torch.float32, 16)
+    assert np.all(np.abs(got - ref) <= TOL * bound), float(np.max(np.abs(got - ref) / np.maximum(bound, 1e-300)))
+    assert device_status() == nv.OK
+
+
+def test_context_bf16_output_repeated_slots(cuda_dev):
+    cache, _, vhat = build_cache(heads=3, chunk=192, fills=[192, 192], seed=17, with_v=True)
+    got, ref, bound = run_context(cache, vhat, [1, 0, 1], [192, 192, 192], 200, 3, torch.bfloat16, 18)
+    assert np.all(np.abs(got - ref) <= TOL * bound + 2.0 ** -8 * np.abs(ref))
+    assert device_status() == nv.OK
+
+
+def test_attention_from_the_cache_end_to_end(cuda_dev):
+    """scores -> softmax (torch, FP32, then bf16 weights) -> context, against attention in
+    float64 on the oracle's K^ and V^: the bf16 weights bound the error (2^-8 of sum p|v|)."""
+    heads, tq = 2, 96
+    cache, khat, vhat = build_cache(heads=heads, chunk=256, fills=[256, 150], seed=19, with_v=True)
+    slots, tokens = [0, 1], [256, 150]
+    tk = 406
+    q = queries(20, tq, heads)
+    scale = 1.0 / np.sqrt(128.0)
+    s_out = torch.empty((heads, tq, 408), dtype=torch.float32, device="cuda")
+    nv.kv_window_scores(cache, slots, tokens, dev_bf16(q), scale, s_out)
+    p = torch.softmax(s_out[:, :, :tk], dim=-1).to(torch.bfloat16)
+    p_full = torch.zeros((heads, tq, 408), dtype=torch.bfloat16, device="cuda")
+    p_full[:, :, :tk] = p
+    o = torch.empty((tq, heads, 128), dtype=torch.float32, device="cuda")
+    nv.kv_window_context(cache, slots, tokens, p_full, o)
+    torch.cuda.synchronize()
+    assert device_status() == nv.OK
+    sref, _ = reference(q, khat, slots, tokens, scale)
+    pref = np.exp(sref - sref.max(axis=-1, keepdims=True))
+    pref /= pref.sum(axis=-1, keepdims=True)
+    vals = synth.bf16_bits_to_f32(np.concatenate([vhat[s][:t] for s, t in zip(slots, tokens)])).astype(np.float64)
+    oref = np.einsum("hij,jhd->ihd", pref, vals)
+    bound = np.einsum("hij,jhd->ihd", pref, np.abs(vals))
+    assert np.all(np.abs(o.cpu().numpy() - oref) <= 2.0 ** -8 * bound + 1e-6)
+
+
+@pytest.mark.slow
+def test_context_full_size_window_sampled_heads(cuda_dev):
+    """24 heads x 128, four chunks of 8192 tokens (32768 keys), 256 queries, FP32 out:
+    heads 0, 11 and 23 checked against the oracle's V^ in full."""
+    heads, chunk = 24, 8192
+    off = synth.kv_offsets(21, heads, 128)
+    cache = nv.KVCache(heads, 128, chunk, 4)
+    vhat = []
+    for s in range(4):
+        k, v = synth.kv_chunk(21, s, chunk, heads, 128, off)
+        nv.kv_quant_append(cache, dev_bf16(k), dev_bf16(v), s)
+        vhat.append(oracle.kv_dequant_chunk(oracle.kv_append(k, v))[1])
+    tk = 4 * chunk
+    pb = weights(22, heads, 256, tk)
+    o = torch.empty((256, heads, 128), dtype=torch.float32, device="cuda")
+    nv.kv_window_context(cache, [0, 1, 2, 3], [chunk] * 4, dev_bf16(pb), o)
+    torch.cuda.synchronize()
+    assert device_status() == nv.OK
+    vals = np.concatenate(vhat)
+    got = o.cpu().numpy().astype(np.float64)
+    for h in (0, 11, 23):
+        pf = synth.bf16_bits_to_f32(pb[h]).astype(np.float64)
+        vf = synth.bf16_bits_to_f32(vals[:, h]).astype(np.float64)
+        ref = pf @ vf
+        bound = pf @ np.abs(vf)
+        assert np.all(np.abs(got[:, h] - ref) <= TOL * bound), f"head {h}"
