@@ -382,6 +382,9 @@ def run_ours(args, rank: int, world: int, local_rank: int):
     s_pair = torch.empty_like(s_fused)
     ko, vo = outs[0].ko, outs[0].vo
 
+    o_fused = torch.empty((SCORES_TQ, HEADS, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+    o_pair = torch.empty((HEADS, SCORES_TQ, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+
     def fused():
         nv.kv_window_scores(cache, win, [CHUNK] * WINDOW, q, 1.0, s_fused)
 
@@ -389,8 +392,16 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         nv.kv_dequant_window(cache, win, ko, vo)
         torch.bmm(q.transpose(0, 1), ko.permute(1, 2, 0), out=s_pair)
 
+    def ctx_fused():  # the V side: weights (here the bf16 scores buffer) times V^ from the cache
+        nv.kv_window_context(cache, win, [CHUNK] * WINDOW, s_fused, o_fused)
+
+    def ctx_pair():
+        nv.kv_dequant_window(cache, win, ko, vo)
+        torch.bmm(s_pair, vo.transpose(0, 1), out=o_pair)
+
     scores = {}
-    for name, fn in (("kv_window_scores", fused), ("window_then_bmm", pair)):
+    for name, fn in (("kv_window_scores", fused), ("window_then_bmm", pair), ("kv_window_context", ctx_fused),
+                     ("window_then_bmm_v", ctx_pair)):
         for _ in range(3):
             fn()
         e0 = torch.cuda.Event(enable_timing=True)
@@ -401,7 +412,7 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         e1.record(stream)
         torch.cuda.synchronize()
         scores[name] = e0.elapsed_time(e1) / 10
-    del s_fused, s_pair
+    del s_fused, s_pair, o_fused, o_pair
     status = nv.get_device_status(local_rank)
     if status != nv.OK:
         raise RuntimeError("device status: " + nv.status_string(status))
@@ -421,12 +432,20 @@ def scores_summary(t, peaks):
     pair_bytes = (WINDOW * 2 * (CHUNK * c // 2 + CHUNK * c // 16) + WINDOW * 2 * 2 * CHUNK * c  # window
                   + keys * c * 2 + SCORES_TQ * c * 2 + HEADS * SCORES_TQ * keys * 2)             # bmm
     gbs = fused_bytes / (t["kv_window_scores"] * 1e-3) / 1e9
-    return {"workload": f"{SCORES_TQ} queries x {HEADS} heads x 128 against {keys} window keys, bf16 scores",
+    # V side: weights [24, tq, keys] bf16 read, V codes and scales read, O written
+    ctx_bytes = HEADS * SCORES_TQ * keys * 2 + keys * c // 2 + keys * c // 16 + SCORES_TQ * c * 2
+    ctx_gbs = ctx_bytes / (t["kv_window_context"] * 1e-3) / 1e9
+    return {"workload": f"{SCORES_TQ} queries x {HEADS} heads x 128 against {keys} window keys, bf16 in/out",
             "kv_window_scores_ms": round(t["kv_window_scores"], 4),
             "window_then_bmm_ms": round(t["window_then_bmm"], 4),
             "speedup": round(t["window_then_bmm"] / t["kv_window_scores"], 3),
             "fused_alg_bytes": fused_bytes, "pair_alg_bytes": pair_bytes,
             "fused_gbs": round(gbs, 1), "fused_frac_hbm": round(gbs / peaks["hbm_gbs"], 3),
+            "kv_window_context_ms": round(t["kv_window_context"], 4),
+            "window_then_bmm_v_ms": round(t["window_then_bmm_v"], 4),
+            "context_speedup": round(t["window_then_bmm_v"] / t["kv_window_context"], 3),
+            "context_alg_bytes": ctx_bytes, "context_gbs": round(ctx_gbs, 1),
+            "context_frac_hbm": round(ctx_gbs / peaks["hbm_gbs"], 3),
             "flops": 2.0 * HEADS * SCORES_TQ * keys * HEAD_DIM}
 
 
@@ -740,7 +759,7 @@ def run_single_kernel(args):
         ko = torch.empty((sum(fills), HEADS, HEAD_DIM), dtype=torch.bfloat16, device=dev)
         vo = torch.empty_like(ko)
         fn = lambda: nv.kv_dequant_window_tokens(cache, list(range(6)), fills, ko, vo)  # noqa: E731
-    elif args.kernel == "kv_scores":
+    elif args.kernel in ("kv_scores", "kv_context"):
         # attention scores of 256 queries x 24 heads against a 4-chunk window, bf16 out
         off = synth.kv_offsets(3, HEADS, HEAD_DIM)
         k, v = synth.kv_chunk(3, 0, CHUNK, HEADS, HEAD_DIM, off)
@@ -752,6 +771,10 @@ def run_single_kernel(args):
         q = to_dev(synth.activations(5, tq, HEADS * HEAD_DIM)).view(tq, HEADS, HEAD_DIM)
         s_out = torch.empty((HEADS, tq, WINDOW * CHUNK), dtype=torch.bfloat16, device=dev)
         fn = lambda: nv.kv_window_scores(cache, list(range(WINDOW)), [CHUNK] * WINDOW, q, 1.0, s_out)  # noqa: E731
+        if args.kernel == "kv_context":
+            nv.kv_window_scores(cache, list(range(WINDOW)), [CHUNK] * WINDOW, q, 1.0 / 128.0, s_out)
+            o = torch.empty((tq, HEADS, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+            fn = lambda: nv.kv_window_context(cache, list(range(WINDOW)), [CHUNK] * WINDOW, s_out, o)  # noqa: E731
     elif args.kernel in ("kv_append", "kv_window"):
         off = synth.kv_offsets(3, HEADS, HEAD_DIM)
         k, v = synth.kv_chunk(3, 0, CHUNK, HEADS, HEAD_DIM, off)
@@ -817,7 +840,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--kernel", default=None,
                     help="profiling mode: gemm | gemm_fused | quantize | dequantize | kv_append | kv_window | kv_window_sink | "
-                         "kv_scores | lora_merge")
+                         "kv_scores | kv_context | lora_merge")
     ap.add_argument("--shape", default="8192,14336,3072", help="M,N,K for gemm; rows,cols for (de)quantize")
     ap.add_argument("--iters", type=int, default=3)
     ap.add_argument("--kernel-warmup", type=int, default=1,
