@@ -356,23 +356,43 @@ __global__ void __launch_bounds__(kThreads, 1)
 // O[i, h, d] = sum_j P[h, i, j] * V^[j, h, d] over the window's keys j, with
 //   V^[j, h, d] = bf16(RN(RN(e2m1 * s) * g_V))   (the window's V, bit for bit)
 // and P given (e.g. the softmax of the scores), FP32 accumulation in tensor memory.
-// CTA (128-query tile, head), 8 warps:
-//   warp 0      TMA producer: P tiles (128 queries x 128 keys bf16, two 64-key boxes,
-//               128-byte swizzle), double-buffered
-//   warp 1      MMA issuer: 8 tcgen05.mma (K = 16 keys each) per key tile into one
-//               128 x 128 FP32 accumulator
-//   warps 4..7  dequantize each key tile's V^ from the cache straight into shared
-//               memory, transposed (128 dims x 128 keys, K-major for the MMA's B
-//               operand), double-buffered; at the end the epilogue (one lane
-//               quarter each): the 128 outputs of a query row, staged in shared
-//               memory and written by TMA stores clipped to the query count.
-constexpr int kCtxThreads = 256;
-constexpr int kCtxBufs = 2;
-constexpr int kPBytes = kQ * kKeys * 2;  // 32 KB
-constexpr int kVBytes = kD * kKeys * 2;  // 32 KB
-constexpr int kCtxSmemBytes = kCtxBufs * (kPBytes + kVBytes) + 1024 /*barriers*/ + 1024 /*alignment*/;
-constexpr int kCtxTmemCols = kD;         // one 128-column accumulator
+// A CTA takes G <= 4 query tiles of 128 queries of one head (G accumulators of 128
+// columns in tensor memory), so each 64-key tile of V^ it dequantizes feeds G tiles of
+// P; a cluster of S CTAs splits the window's key tiles into S contiguous ranges.  The
+// host picks G and S for the fewest waves of the longest CTA.  12 warps:
+//   warp 0      TMA producer: per key tile, G boxes of P (128 queries x 64 keys bf16,
+//               128-byte swizzle), two stages
+//   warp 1      MMA issuer: per key tile and query tile, 4 tcgen05.mma (K = 16 keys)
+//   warps 4..11 dequantize each key tile's V^ into shared memory transposed (128 dims
+//               x 64 keys: the MMA's K-major B operand), two buffers.  Each thread
+//               copies the code words, scale word and g_V of its two keys into a
+//               private ring of shared memory with cp.async, kRing - 1 tiles ahead of
+//               the tile it decodes.  Warps 4..7 (one lane quarter each) then read the
+//               accumulators.
+// With S = 1 the accumulators go straight to the output.  With S > 1, query tile by
+// query tile, every CTA puts its partial in shared memory and CTA r sums rows
+// [128 r / S, 128 (r + 1) / S) over the cluster in rank order (distributed shared
+// memory; a fixed order, so the result does not depend on scheduling).
+constexpr int kCtxThreads = 384;
+constexpr int kCtxKeys = 64;                          // keys per tile (K of 4 MMAs)
+constexpr int kCtxMaxG = 4;                           // query tiles per CTA
+constexpr int kPTileBytes = kQ * kCtxKeys * 2;        // 16 KB: 128 queries x 64 keys
+constexpr int kPStageBytes = kCtxMaxG * kPTileBytes;  // 64 KB
+constexpr int kCtxPBufs = 2;
+constexpr int kVTBytes = kD * kCtxKeys * 2;           // 16 KB: 128 dims x 64 keys
+constexpr int kCtxVBufs = 2;
 constexpr int kVWarp0 = 4;
+constexpr int kVThreads = 256;                        // warps 4..11
+constexpr int kRing = 6;                              // key tiles of V cache data in flight
+// per ring stage and decoder thread, for its two keys: 8 code bytes, the 4-byte word
+// holding the scale byte, g_V
+constexpr int kRingStageBytes = 2 * kVThreads * (8 + 4 + 4);
+constexpr int kPartRowBytes = kD * 4;                 // one query row of an FP32 partial
+constexpr int kCtxSmemBytes = kCtxPBufs * kPStageBytes + kCtxVBufs * kVTBytes + kRing * kRingStageBytes +
+                              1024 /*barriers*/ + 1024 /*alignment*/;
+static_assert(kCtxPBufs * kPStageBytes >= kQ * kPartRowBytes, "a partial tile reuses the P stages");
+constexpr int kCtxTmemCols = kCtxMaxG * kD;           // 512
+constexpr int kMaxSplit = 8;
 
 struct ContextParams {
   const uint8_t* base;
@@ -383,45 +403,110 @@ struct ContextParams {
   int32_t tokens[kMaxWindowSlots];
   int64_t key_end[kMaxWindowSlots];
   int64_t Tq, Tk;
+  int64_t tiles_per_split;  // key tiles per CTA of a cluster
+  int32_t split;            // S: CTAs per (query group, head) = cluster size
+  int32_t G;                // query tiles per CTA
+  int32_t n_qt;             // query tiles in all
   bool o_bf16;
+  uint8_t* o;
+  int64_t ldo;
   unsigned* status;
   unsigned long long wait_limit_ns;
 };
 
+// Copy one key's 16 dims of V (8 code bytes; the 4-byte word holding its scale byte)
+// from the cache into this thread's ring slot and store its g_V there; keys beyond the
+// window or in a slot that holds another count are zero-filled (they decode to +0).
+__device__ __forceinline__ void ctx_issue(const ContextParams& p, const int32_t* valid, const float* gv_tab,
+                                          int64_t j, int h, int dq, int& seg, uint32_t dst_codes,
+                                          uint32_t dst_scales, float* dst_gv) {
+  const uint8_t* src_c = p.base;
+  const uint8_t* src_s = p.base;
+  uint32_t n = 0;
+  float gv = 0.0f;
+  if (j < p.Tk) {
+    while (j >= p.key_end[seg]) ++seg;  // keys only grow along a CTA's range
+    if (valid[seg]) {
+      const int slot = p.slots[seg];
+      const int64_t tok = j - (seg == 0 ? 0 : p.key_end[seg - 1]);
+      const int64_t el = (tok * p.heads + h) * kD + dq * 16;  // element within the slot
+      src_c = p.base + p.off_v_codes + slot * p.slot_codes_bytes + el / 2;
+      src_s = p.base + p.off_v_scales + slot * p.slot_scales_bytes + ((el / 16) & ~int64_t(3));
+      n = 8;
+      gv = gv_tab[seg];
+    }
+  }
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst_codes), "l"(src_c), "r"(n) : "memory");
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(dst_scales), "l"(src_s), "r"(n >> 1)
+               : "memory");
+  *dst_gv = gv;
+}
+
+// 16 dims of one key as floats: e2m1 * s exactly (f16), then one FP32 product with g_V.
+__device__ __forceinline__ void ctx_decode(uint32_t w0, uint32_t w1, uint32_t sbyte, float gv, float (&f)[16]) {
+  const uint32_t s2 = e4m3_to_f16x2_bcast(sbyte);
+  uint32_t h0[4], h1[4];
+  e2m1x8_times_scale(w0, s2, h0);  // dims 0..7
+  e2m1x8_times_scale(w1, s2, h1);  // dims 8..15
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float lo, hi;
+    f16x2_to_f32x2(h0[q], lo, hi);  // e2m1 * s, exact
+    mul2(f[2 * q], f[2 * q + 1], lo, hi, gv, gv);
+    f16x2_to_f32x2(h1[q], lo, hi);
+    mul2(f[8 + 2 * q], f[9 + 2 * q], lo, hi, gv, gv);
+  }
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
+}
+
 // kind::f16 again (M = N = 128); the B operand is V^ transposed (dims x keys).
 __global__ void __launch_bounds__(kCtxThreads, 1)
-    kv_context_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ CUtensorMap map_o,
-                      ContextParams p) {
+    kv_context_kernel(const __grid_constant__ CUtensorMap map_p, const __grid_constant__ ContextParams p) {
   pdl_trigger();
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* pbuf = smem;                                // kCtxBufs P tiles
-  uint8_t* vbuf = smem + kCtxBufs * kPBytes;           // kCtxBufs V^T tiles
-  uint8_t* bar_area = vbuf + kCtxBufs * kVBytes;
+  uint8_t* pbuf = smem;                                // P stages; the partial output at the end
+  uint8_t* vbuf = smem + kCtxPBufs * kPStageBytes;     // V^T tiles
+  uint8_t* ring = vbuf + kCtxVBufs * kVTBytes;         // V cache data in flight
+  uint8_t* bar_area = ring + kRing * kRingStageBytes;
   uint64_t* p_full = reinterpret_cast<uint64_t*>(bar_area);
-  uint64_t* p_empty = p_full + kCtxBufs;
-  uint64_t* v_full = p_empty + kCtxBufs;
-  uint64_t* v_empty = v_full + kCtxBufs;
-  uint64_t* t_full = v_empty + kCtxBufs;
+  uint64_t* p_empty = p_full + kCtxPBufs;
+  uint64_t* v_full = p_empty + kCtxPBufs;
+  uint64_t* v_empty = v_full + kCtxVBufs;
+  uint64_t* t_full = v_empty + kCtxVBufs;
   uint64_t* done_bar = t_full + 1;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(done_bar + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int32_t* valid = reinterpret_cast<int32_t*>(tmem_slot + 2);         // per list entry: its slot holds the count
+  float* gv_tab = reinterpret_cast<float*>(valid + kMaxWindowSlots);  // per list entry: g_V of its slot
+  volatile int* acc_ok = reinterpret_cast<volatile int*>(gv_tab + kMaxWindowSlots);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int qt = blockIdx.x, h = blockIdx.y;
-  const int64_t n_kt = (p.Tk + kKeys - 1) / kKeys;
+  const int rank = blockIdx.x, qg = blockIdx.y, h = blockIdx.z;  // rank = this CTA's rank in its cluster
+  const int qt0 = qg * p.G;
+  const int G = p.n_qt - qt0 < p.G ? p.n_qt - qt0 : p.G;         // this CTA's query tiles
+  const int64_t n_kt = (p.Tk + kCtxKeys - 1) / kCtxKeys;
+  const int64_t kt0 = rank * p.tiles_per_split;
+  const int64_t kt_end = kt0 + p.tiles_per_split < n_kt ? kt0 + p.tiles_per_split : n_kt;
+  const uint32_t n_my = kt_end > kt0 ? (uint32_t)(kt_end - kt0) : 0u;
   const unsigned long long limit = p.wait_limit_ns;
 
   if (threadIdx.x == 0) {
-    for (int b = 0; b < kCtxBufs; ++b) {
+    for (int b = 0; b < kCtxPBufs; ++b) {
       mbar_init(smem_u32(&p_full[b]), 1);
       mbar_init(smem_u32(&p_empty[b]), 1);
-      mbar_init(smem_u32(&v_full[b]), 4);
+    }
+    for (int b = 0; b < kCtxVBufs; ++b) {
+      mbar_init(smem_u32(&v_full[b]), kVThreads / 32);
       mbar_init(smem_u32(&v_empty[b]), 1);
     }
     mbar_init(smem_u32(t_full), 1);
     mbar_init(smem_u32(done_bar), 1);
     *abort_flag = 0;
+    *acc_ok = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   if (warp == 0) {
@@ -430,11 +515,18 @@ __global__ void __launch_bounds__(kCtxThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  pdl_wait();  // the cache and P come from earlier work
+  if (threadIdx.x < p.n_slots) {
+    const int i = threadIdx.x;
+    const bool ok = reinterpret_cast<const int32_t*>(p.base + p.off_tokens)[p.slots[i]] == p.tokens[i];
+    valid[i] = ok ? 1 : 0;
+    gv_tab[i] = reinterpret_cast<const float*>(p.base + p.off_gscale)[2 * p.slots[i] + 1];
+    if (!ok && rank == 0) set_status(p.status, kStatusShape);  // the slot holds another token count
+  }
   fence_before();
   __syncthreads();
   fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();  // the cache and P come from earlier work
 
   if (warp == 0) {
     // ------------------------------------------------------------ P producer
@@ -442,48 +534,47 @@ __global__ void __launch_bounds__(kCtxThreads, 1)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_p)) : "memory");
       bool ok = true;
       uint32_t issued = 0;
-      for (uint32_t kt = 0; kt < (uint32_t)n_kt; ++kt) {
-        const int b = kt % kCtxBufs;
-        if (!mbar_wait(smem_u32(&p_empty[b]), ((kt / kCtxBufs) & 1u) ^ 1u, abort_flag, limit)) {
+      for (uint32_t i = 0; i < n_my; ++i) {
+        const int b = i % kCtxPBufs;
+        if (!mbar_wait(smem_u32(&p_empty[b]), ((i / kCtxPBufs) & 1u) ^ 1u, abort_flag, limit)) {
           ok = false;
           break;
         }
         const uint32_t fb = smem_u32(&p_full[b]);
-        mbar_arrive_expect_tx(fb, kPBytes);
-        uint8_t* dst = pbuf + b * kPBytes;
-        tma_load_3d(smem_u32(dst), &map_p, fb, (int32_t)(kt * kKeys), qt * kQ, h);
-        tma_load_3d(smem_u32(dst + kBlockBytes), &map_p, fb, (int32_t)(kt * kKeys + 64), qt * kQ, h);
-        issued = kt + 1;
+        mbar_arrive_expect_tx(fb, (uint32_t)(G * kPTileBytes));
+        const int32_t key = (int32_t)((kt0 + i) * kCtxKeys);
+        for (int g = 0; g < G; ++g)
+          tma_load_3d(smem_u32(pbuf + b * kPStageBytes + g * kPTileBytes), &map_p, fb, key, (qt0 + g) * kQ, h);
+        issued = i + 1;
       }
       if (!ok) {
         set_status(p.status, kStatusTimeout);
         *abort_flag = 1;
       }
-      for (uint32_t j = issued > (uint32_t)kCtxBufs ? issued - kCtxBufs : 0; j < issued; ++j)
-        mbar_wait_drain(smem_u32(&p_full[j % kCtxBufs]), (j / kCtxBufs) & 1u, limit);
+      for (uint32_t j = issued > (uint32_t)kCtxPBufs ? issued - kCtxPBufs : 0; j < issued; ++j)
+        mbar_wait_drain(smem_u32(&p_full[j % kCtxPBufs]), (j / kCtxPBufs) & 1u, limit);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       bool ok = true;
-      for (uint32_t kt = 0; kt < (uint32_t)n_kt; ++kt) {
-        const int b = kt % kCtxBufs;
-        const uint32_t ph = (kt / kCtxBufs) & 1u;
-        if (!mbar_wait(smem_u32(&v_full[b]), ph, abort_flag, limit) ||
-            !mbar_wait(smem_u32(&p_full[b]), ph, abort_flag, limit)) {
+      for (uint32_t i = 0; i < n_my; ++i) {
+        const int bp = i % kCtxPBufs, bv = i % kCtxVBufs;
+        if (!mbar_wait(smem_u32(&v_full[bv]), (i / kCtxVBufs) & 1u, abort_flag, limit) ||
+            !mbar_wait(smem_u32(&p_full[bp]), (i / kCtxPBufs) & 1u, abort_flag, limit)) {
           ok = false;
           break;
         }
         fence_after();
-        const uint32_t a_addr = smem_u32(pbuf + b * kPBytes), b_addr = smem_u32(vbuf + b * kVBytes);
+        const uint32_t a_addr = smem_u32(pbuf + bp * kPStageBytes), b_addr = smem_u32(vbuf + bv * kVTBytes);
+        for (int g = 0; g < G; ++g) {
 #pragma unroll
-        for (int kk = 0; kk < kKeys / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * kBlockBytes + (kk & 3) * 32;
-          mma_bf16(tmem_base, smem_desc(a_addr + off, 16, 1024, 2), smem_desc(b_addr + off, 16, 1024, 2),
-                   (kt > 0 || kk > 0) ? 1u : 0u);
+          for (int kk = 0; kk < kCtxKeys / 16; ++kk)
+            mma_bf16(tmem_base + (uint32_t)(g * kD), smem_desc(a_addr + g * kPTileBytes + kk * 32, 16, 1024, 2),
+                     smem_desc(b_addr + kk * 32, 16, 1024, 2), (i > 0 || kk > 0) ? 1u : 0u);
         }
-        commit(smem_u32(&p_empty[b]));
-        commit(smem_u32(&v_empty[b]));
+        commit(smem_u32(&p_empty[bp]));
+        commit(smem_u32(&v_empty[bv]));
       }
       if (!ok) {
         set_status(p.status, kStatusTimeout);
@@ -495,128 +586,178 @@ __global__ void __launch_bounds__(kCtxThreads, 1)
       mbar_wait_drain(smem_u32(done_bar), 0, limit);
     }
   } else if (warp >= kVWarp0) {
-    // ------------------------------------------------------------ V^T producers, then epilogue
-    const int t = threadIdx.x - kVWarp0 * 32;  // 0..127
-    const int kp = t & 63;                     // key pair of the tile: keys 2 kp, 2 kp + 1
-    const int dh = t >> 6;                     // dims [64 dh, 64 dh + 64)
+    // ------------------------------------------------------------ V^T producers
+    const int t = threadIdx.x - kVWarp0 * 32;  // 0..255
+    const int kp = t & 31;                     // key pair of the tile: keys 2 kp, 2 kp + 1
+    const int dq = t >> 5;                     // dims [16 dq, 16 dq + 16) (one scale block)
+    const int col = 2 * kp;                    // key within the tile (even)
+    int seg0 = 0, seg1 = 0;
+    // ring stage st: codes [2][kVThreads] x 8 B, scale words [2][kVThreads] x 4 B, g_V
+    // [2][kVThreads] x 4 B; this thread's entries only
+    auto codes_at = [&](int st, int e) { return smem_u32(ring + st * kRingStageBytes + (e * kVThreads + t) * 8); };
+    auto scales_at = [&](int st, int e) {
+      return smem_u32(ring + st * kRingStageBytes + 2 * kVThreads * 8 + (e * kVThreads + t) * 4);
+    };
+    auto gv_at = [&](int st, int e) {
+      return reinterpret_cast<float*>(ring + st * kRingStageBytes + 2 * kVThreads * 12 + (e * kVThreads + t) * 4);
+    };
+    auto issue = [&](uint32_t i) {
+      const int st = i % kRing;
+      const int64_t j = (kt0 + i) * kCtxKeys + col;
+      ctx_issue(p, valid, gv_tab, j, h, dq, seg0, codes_at(st, 0), scales_at(st, 0), gv_at(st, 0));
+      ctx_issue(p, valid, gv_tab, j + 1, h, dq, seg1, codes_at(st, 1), scales_at(st, 1), gv_at(st, 1));
+    };
+    for (uint32_t i = 0; i + 1 < (uint32_t)kRing; ++i) {
+      if (i < n_my) issue(i);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+    }
+    const int sh = 8 * (dq & 3);  // this thread's scale byte within the word
+    // row d of a V^T tile holds its 64 keys (128 bytes, 16-byte chunks swizzled by d % 8);
+    // keys 2 kp and 2 kp + 1 share one 32-bit word
+    const uint32_t vt_off = (uint32_t)((col & 7) * 2);
+    const uint32_t chunk = (uint32_t)(col >> 3);
     bool ok = true;
-    for (uint32_t kt = 0; kt < (uint32_t)n_kt && ok; ++kt) {
-      const int b = kt % kCtxBufs;
-      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&v_empty[b]), ((kt / kCtxBufs) & 1u) ^ 1u, abort_flag,
+    for (uint32_t i = 0; i < n_my; ++i) {
+      if (i + kRing - 1 < n_my) issue(i + kRing - 1);
+      asm volatile("cp.async.commit_group;" ::: "memory");
+      asm volatile("cp.async.wait_group %0;" ::"n"(kRing - 1) : "memory");
+      const int st = i % kRing;
+      float f0[16], f1[16];
+      {
+        uint32_t a0, a1, b0, b1, s0, s1;
+        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(a0), "=r"(a1) : "r"(codes_at(st, 0)));
+        asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(codes_at(st, 1)));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(s0) : "r"(scales_at(st, 0)));
+        asm volatile("ld.shared.u32 %0, [%1];" : "=r"(s1) : "r"(scales_at(st, 1)));
+        ctx_decode(a0, a1, (s0 >> sh) & 0xFFu, *gv_at(st, 0), f0);
+        ctx_decode(b0, b1, (s1 >> sh) & 0xFFu, *gv_at(st, 1), f1);
+      }
+      const int b = i % kCtxVBufs;
+      if (!__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(&v_empty[b]), ((i / kCtxVBufs) & 1u) ^ 1u, abort_flag,
                                              limit))) {
         ok = false;
         break;
       }
       fence_after();
-      // the 64 dims of each of the two keys, decoded to bf16 (zeros beyond the window)
-      uint32_t vals[2][32];  // [key][dim pair] as bf16x2 along dims
+      const uint32_t vb = smem_u32(vbuf + b * kVTBytes) + (uint32_t)(dq * 16 * 128) + vt_off;
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int64_t j = (int64_t)kt * kKeys + 2 * kp + e;
-        int32_t slot = -1;
-        int64_t tok = 0;
-        if (j < p.Tk) {
-          int i = 0;
-          while (j >= p.key_end[i]) ++i;
-          const int64_t begin = i == 0 ? 0 : p.key_end[i - 1];
-          if (reinterpret_cast<const int32_t*>(p.base + p.off_tokens)[p.slots[i]] == p.tokens[i]) {
-            slot = p.slots[i];
-            tok = j - begin;
-          } else if (j == begin) {
-            set_status(p.status, kStatusShape);  // the slot holds another token count
-          }
-        }
-#pragma unroll
-        for (int q = 0; q < 32; ++q) vals[e][q] = 0;
-        if (slot >= 0) {
-          const int64_t el = (tok * p.heads + h) * kD + dh * 64;  // element within the slot
-          const uint8_t* cp = p.base + p.off_v_codes + slot * p.slot_codes_bytes + el / 2;
-          const uint4 c0 = *reinterpret_cast<const uint4*>(cp), c1 = *reinterpret_cast<const uint4*>(cp + 16);
-          const uint32_t sc4 = *reinterpret_cast<const uint32_t*>(p.base + p.off_v_scales + slot * p.slot_scales_bytes + el / 16);
-          const float gv = reinterpret_cast<const float*>(p.base + p.off_gscale)[2 * slot + 1];
-          const uint32_t cw[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-#pragma unroll
-          for (int g8 = 0; g8 < 8; ++g8) {  // 8 dims per code word, 16 per scale byte
-            uint32_t hv[4];
-            e2m1x8_times_scale(cw[g8], e4m3_to_f16x2_bcast((sc4 >> (8 * (g8 >> 1))) & 0xFFu), hv);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              float lo, hi;
-              f16x2_to_f32x2(hv[q], lo, hi);  // e2m1 * s, exact
-              vals[e][g8 * 4 + q] = pack_bf16x2(lo * gv, hi * gv);
-            }
-          }
-        }
-      }
-      // transposed store: row d holds keys along the row; one 32-bit store carries keys
-      // 2 kp and 2 kp + 1 of dim d (128-byte swizzle on 16-byte chunks)
-      uint8_t* vb = vbuf + b * kVBytes;
-      const int col = 2 * kp;                 // key within the tile (even)
-      const int blk = col >> 6, cb = col & 63;
-#pragma unroll
-      for (int q = 0; q < 32; ++q) {
-#pragma unroll
-        for (int e2 = 0; e2 < 2; ++e2) {      // dims 2 q and 2 q + 1 of this half
-          const int d = dh * 64 + 2 * q + e2;
-          const uint32_t lo = e2 ? (vals[0][q] >> 16) : (vals[0][q] & 0xFFFFu);
-          const uint32_t hi = e2 ? (vals[1][q] >> 16) : (vals[1][q] & 0xFFFFu);
-          *reinterpret_cast<uint32_t*>(vb + blk * kBlockBytes + d * 128 + ((((cb >> 3) ^ (d & 7))) << 4) +
-                                       (cb & 7) * 2) = lo | (hi << 16);
-        }
-      }
+      for (int d = 0; d < 16; ++d)  // dim 16 dq + d; (16 dq + d) % 8 = d % 8
+        asm volatile("st.shared.u32 [%0], %1;" ::"r"(vb + (uint32_t)(d * 128) + ((chunk ^ (uint32_t)(d & 7)) << 4)),
+                     "r"(pack_bf16x2(f0[d], f1[d]))
+                     : "memory");
       fence_proxy_async_smem();  // the tensor core reads V^T through the async proxy
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&v_full[b]));
     }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // no copy into the ring outlives the loop
     if (!ok) {
       if (lane == 0) set_status(p.status, kStatusTimeout);
       *abort_flag = 1;
-    } else {
-      // epilogue: warp w reads tensor-memory lane quarter w % 4 (query rows 32 (w % 4) ..)
-      const int quarter = warp & 3;
+    } else if (warp < kVWarp0 + 4) {
       if (__all_sync(0xFFFFFFFFu, mbar_wait(smem_u32(t_full), 0, abort_flag, limit))) {
-        fence_after();
-        // the P buffers are free once every MMA has completed: 8 KB of staging per warp
-        const uint32_t wbuf = smem_u32(pbuf) + (uint32_t)((warp - kVWarp0) * 2 * kBoxBytes);
-        const int cols = p.o_bf16 ? 64 : 32;
-        uint32_t nbox = 0;
-        for (int c0 = 0; c0 < kD; c0 += cols, ++nbox) {
-          uint32_t w[32];
-          {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + c0, r);
-            if (p.o_bf16) {
-#pragma unroll
-              for (int i = 0; i < 16; ++i) w[i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-              tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + c0 + 32, r);
-#pragma unroll
-              for (int i = 0; i < 16; ++i)
-                w[16 + i] = pack_bf16x2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-            } else {
-#pragma unroll
-              for (int i = 0; i < 32; ++i) w[i] = r[i];
-            }
-          }
-          const uint32_t buf = wbuf + (nbox & 1u) * kBoxBytes;
-          if (lane == 0) asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory");
-          __syncwarp();
-#pragma unroll
-          for (int c = 0; c < 8; ++c)
-            st_shared_v4(buf + lane * 128 + ((c ^ (lane & 7)) << 4),
-                         make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]));
-          fence_proxy_async_smem();
-          __syncwarp();
-          if (lane == 0) {
-            tma_store_2d(&map_o, buf, h * kD + c0, qt * kQ + quarter * 32);
-            asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-          }
-        }
-        if (lane == 0) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
-        __syncwarp();
+        if (warp == kVWarp0 && lane == 0) *acc_ok = 1;
       } else {
         if (lane == 0) set_status(p.status, kStatusTimeout);
         *abort_flag = 1;
       }
+    }
+  }
+
+  fence_before();
+  __syncthreads();
+  fence_after();
+
+  // ---------------------------------------------------------------- output
+  // warps 4..7: warp w reads tensor-memory lane quarter w % 4 (query rows 32 (w % 4) ..)
+  const bool reader = warp >= kVWarp0 && warp < kVWarp0 + 4;
+  const int quarter = warp & 3;
+  const bool have = *acc_ok != 0 && n_my > 0;
+  if (p.split == 1) {
+    if (reader && *acc_ok) {
+      for (int g = 0; g < G; ++g) {
+        const int64_t qrow = (int64_t)(qt0 + g) * kQ + quarter * 32 + lane;
+#pragma unroll 1
+        for (int c0 = 0; c0 < kD; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * kD + c0), r);
+          if (qrow < p.Tq) {
+            if (p.o_bf16) {
+              uint4* dst = reinterpret_cast<uint4*>(p.o + (qrow * p.ldo + (int64_t)h * kD + c0) * 2);
+#pragma unroll
+              for (int k = 0; k < 4; ++k)
+                dst[k] = make_uint4(pack_bf16x2(__uint_as_float(r[8 * k]), __uint_as_float(r[8 * k + 1])),
+                                    pack_bf16x2(__uint_as_float(r[8 * k + 2]), __uint_as_float(r[8 * k + 3])),
+                                    pack_bf16x2(__uint_as_float(r[8 * k + 4]), __uint_as_float(r[8 * k + 5])),
+                                    pack_bf16x2(__uint_as_float(r[8 * k + 6]), __uint_as_float(r[8 * k + 7])));
+            } else {
+              uint4* dst = reinterpret_cast<uint4*>(p.o + (qrow * p.ldo + (int64_t)h * kD + c0) * 4);
+#pragma unroll
+              for (int k = 0; k < 8; ++k) dst[k] = make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]);
+            }
+          }
+        }
+      }
+    }
+  } else {
+    const int r0 = rank * kQ / p.split, r1 = (rank + 1) * kQ / p.split;
+    const uint32_t part = smem_u32(pbuf);
+    for (int g = 0; g < G; ++g) {  // the same G in every CTA of the cluster
+      if (reader) {
+        // partial -> shared memory: row r's 16-byte chunks XOR-swizzled by r % 32
+        const int row = quarter * 32 + lane;
+        const uint32_t prow = part + (uint32_t)(row * kPartRowBytes);
+#pragma unroll 1
+        for (int c0 = 0; c0 < kD; c0 += 32) {
+          uint32_t r[32];
+          if (have) {
+            tmem_ld_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(g * kD + c0), r);
+          } else {
+#pragma unroll
+            for (int k = 0; k < 32; ++k) r[k] = 0u;  // no keys in this CTA's range (or a timeout)
+          }
+#pragma unroll
+          for (int k = 0; k < 8; ++k)
+            st_shared_v4(prow + ((((c0 >> 2) + k) ^ lane) << 4),
+                         make_uint4(r[4 * k], r[4 * k + 1], r[4 * k + 2], r[4 * k + 3]));
+        }
+      }
+      __syncthreads();
+      cluster_sync_all();  // every CTA of the cluster has this tile's partial in shared memory
+      for (int it = threadIdx.x; it < (r1 - r0) * (kD / 8); it += kCtxThreads) {
+        const int r = r0 + it / (kD / 8), cg = it % (kD / 8);  // 8 output columns 8 cg ..
+        const uint32_t a0 = part + (uint32_t)(r * kPartRowBytes) + ((uint32_t)((2 * cg) ^ (r & 31)) << 4);
+        const uint32_t a1 = part + (uint32_t)(r * kPartRowBytes) + ((uint32_t)((2 * cg + 1) ^ (r & 31)) << 4);
+        float acc[8];
+        for (int src = 0; src < p.split; ++src) {  // cluster-rank order
+          float v[8];
+          uint32_t b0, b1;
+          asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(b0) : "r"(a0), "r"(src));
+          asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(b1) : "r"(a1), "r"(src));
+          asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+                       : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
+                       : "r"(b0)
+                       : "memory");
+          asm volatile("ld.shared::cluster.v4.f32 {%0,%1,%2,%3}, [%4];"
+                       : "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+                       : "r"(b1)
+                       : "memory");
+#pragma unroll
+          for (int k = 0; k < 8; ++k) acc[k] = src == 0 ? v[k] : __fadd_rn(acc[k], v[k]);
+        }
+        const int64_t qrow = (int64_t)(qt0 + g) * kQ + r;
+        if (qrow < p.Tq) {
+          if (p.o_bf16) {
+            *reinterpret_cast<uint4*>(p.o + (qrow * p.ldo + (int64_t)h * kD + cg * 8) * 2) =
+                make_uint4(pack_bf16x2(acc[0], acc[1]), pack_bf16x2(acc[2], acc[3]), pack_bf16x2(acc[4], acc[5]),
+                           pack_bf16x2(acc[6], acc[7]));
+          } else {
+            float4* dst = reinterpret_cast<float4*>(p.o + (qrow * p.ldo + (int64_t)h * kD + cg * 8) * 4);
+            dst[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
+            dst[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
+          }
+        }
+      }
+      cluster_sync_all();  // no CTA rewrites or releases its partial while another reads it
     }
   }
 
@@ -752,6 +893,8 @@ cudaError_t launch_kv_context(const KVLayout& L, const int32_t* slots, const int
   p.Tq = tq;
   p.Tk = acc;
   p.o_bf16 = o_bf16;
+  p.o = static_cast<uint8_t*>(o_out);
+  p.ldo = ldo;
   p.status = status;
   p.wait_limit_ns = kWaitLimitNs;
   if (tq == 0) return cudaSuccess;
@@ -768,28 +911,82 @@ cudaError_t launch_kv_context(const KVLayout& L, const int32_t* slots, const int
          CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
-  // O [tq][heads * 128] (row pitch ldo): 32-row x 128-byte boxes, clipped at tq rows
-  CUtensorMap mo;
-  const cuuint64_t esz = o_bf16 ? 2 : 4;
-  cuuint64_t odims[2] = {(cuuint64_t)L.heads * kD, (cuuint64_t)tq};
-  cuuint64_t ostrides[1] = {(cuuint64_t)ldo * esz};
-  cuuint32_t obox[2] = {(cuuint32_t)(128 / esz), 32};
-  if (fn(&mo, o_bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, o_out, odims,
-         ostrides, obox, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
-    return cudaErrorInvalidValue;
-  static std::atomic<bool> done[64];
+
+  // per device: shared-memory opt-in once, and how many CTAs can be resident at once in
+  // clusters of S = 1 .. kMaxSplit (0: that cluster size cannot be resident)
+  static std::atomic<int> conc_cache[64][kMaxSplit + 1];
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
-  if (!done[dev].load(std::memory_order_relaxed)) {
+  if (conc_cache[dev][0].load(std::memory_order_relaxed) == 0) {
     e = cudaFuncSetAttribute(kv_context_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kCtxSmemBytes);
     if (e != cudaSuccess) return e;
-    done[dev].store(true, std::memory_order_relaxed);
+    for (int c = 1; c <= kMaxSplit; ++c) {
+      cudaLaunchConfig_t cfg = {};
+      cfg.gridDim = dim3((unsigned)c, 1, 1);
+      cfg.blockDim = dim3(kCtxThreads, 1, 1);
+      cfg.dynamicSmemBytes = kCtxSmemBytes;
+      cudaLaunchAttribute attr;
+      attr.id = cudaLaunchAttributeClusterDimension;
+      attr.val.clusterDim.x = (unsigned)c;
+      attr.val.clusterDim.y = 1;
+      attr.val.clusterDim.z = 1;
+      cfg.attrs = &attr;
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kv_context_kernel, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+      }
+      if (c == 1 && n <= 0) return cudaErrorInvalidConfiguration;
+      conc_cache[dev][c].store(n * c, std::memory_order_relaxed);
+    }
+    conc_cache[dev][0].store(1, std::memory_order_relaxed);
   }
-  const dim3 grid((unsigned)((tq + kQ - 1) / kQ), (unsigned)L.heads, 1);
-  launch_pdl(kv_context_kernel, grid, kCtxThreads, kCtxSmemBytes, s, mp, mo, p);
+  // G query tiles per CTA and S CTAs per cluster: the fewest waves of CTAs times the
+  // longest CTA's work, in units of one P tile (128 queries x 64 keys) with a V^ tile's
+  // dequantization counted as half of one.  Ties keep the smaller S.
+  const int64_t n_kt = (acc + kCtxKeys - 1) / kCtxKeys;
+  const int64_t n_qt = (tq + kQ - 1) / kQ;
+  int best_g = 1, best_s = 1;
+  double best = -1.0;
+  for (int g = 1; g <= kCtxMaxG && g <= n_qt; ++g) {
+    for (int sp = 1; sp <= kMaxSplit && sp <= n_kt; ++sp) {
+      const int64_t conc = conc_cache[dev][sp].load(std::memory_order_relaxed);
+      if (conc <= 0) continue;
+      const int64_t ctas = (int64_t)sp * ((n_qt + g - 1) / g) * L.heads;
+      const int64_t waves = (ctas + conc - 1) / conc;
+      const double cost = (double)waves * (double)((n_kt + sp - 1) / sp) * (g + 0.5);
+      if (best < 0.0 || cost < best * (1.0 - 1e-9)) {
+        best = cost;
+        best_g = g;
+        best_s = sp;
+      }
+    }
+  }
+  const int split = best_s;
+  p.split = split;
+  p.G = best_g;
+  p.n_qt = (int32_t)n_qt;
+  p.tiles_per_split = (n_kt + split - 1) / split;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)split, (unsigned)((n_qt + best_g - 1) / best_g), (unsigned)L.heads);
+  cfg.blockDim = dim3(kCtxThreads, 1, 1);
+  cfg.dynamicSmemBytes = kCtxSmemBytes;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)split;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  e = cudaLaunchKernelEx(&cfg, kv_context_kernel, mp, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

@@ -196,6 +196,34 @@ def test_context_bf16_output_repeated_slots(cuda_dev):
     assert device_status() == nv.OK
 
 
+@pytest.mark.parametrize("heads,chunk,fills,slots,tokens,tq,dtype", [
+    # 16 key tiles: the keys of each (query tile, head) split over a cluster of two CTAs
+    (2, 1024, [1024, 1000], [1, 0], [1000, 1024], 130, torch.float32),
+    # 72 key tiles (slot boundaries inside tiles): eight CTAs, the last range ragged
+    (1, 4096, [4096, 4096, 900], [2, 0, 1], [900, 4096, 4096], 70, torch.bfloat16),
+])
+def test_context_keys_split_across_a_cluster(cuda_dev, heads, chunk, fills, slots, tokens, tq, dtype):
+    """Few query tiles against many keys: the partial outputs of the CTAs of a cluster are
+    summed over distributed shared memory; the result stays within the FP32 bound."""
+    cache, _, vhat = build_cache(heads=heads, chunk=chunk, fills=fills, seed=23, with_v=True)
+    device_status(clear=True)
+    got, ref, bound = run_context(cache, vhat, slots, tokens, tq, heads, dtype, 24)
+    extra = 2.0 ** -8 * np.abs(ref) if dtype == torch.bfloat16 else 0.0
+    assert np.all(np.abs(got - ref) <= TOL * bound + extra)
+    assert device_status() == nv.OK
+
+
+def test_context_wrong_token_count_sets_shape_status(cuda_dev):
+    cache, _, _ = build_cache(heads=1, chunk=2048, fills=[2048, 100], seed=25, with_v=True)
+    p = torch.zeros((1, 8, 4096), dtype=torch.bfloat16, device="cuda")
+    o = torch.empty((8, 1, 128), dtype=torch.float32, device="cuda")
+    device_status(clear=True)
+    nv.kv_window_context(cache, [0, 1], [2048, 2048], p, o)  # slot 1 holds 100 tokens
+    torch.cuda.synchronize()
+    assert device_status() == nv.ERR_SHAPE
+    assert torch.all(o == 0)  # its keys are read as zeros
+
+
 def test_attention_from_the_cache_end_to_end(cuda_dev):
     """scores -> softmax (torch, FP32, then bf16 weights) -> context, against attention in
     float64 on the oracle's K^ and V^: the bf16 weights bound the error (2^-8 of sum p|v|)."""
