@@ -760,14 +760,15 @@ def run_single_kernel(args):
         vo = torch.empty_like(ko)
         fn = lambda: nv.kv_dequant_window_tokens(cache, list(range(6)), fills, ko, vo)  # noqa: E731
     elif args.kernel in ("kv_scores", "kv_context"):
-        # attention scores of 256 queries x 24 heads against a 4-chunk window, bf16 out
+        # attention scores (or outputs) of SCORES_TQ queries x 24 heads against a 4-chunk
+        # window, bf16 out: the workload of the attention-side measurement of the step run
         off = synth.kv_offsets(3, HEADS, HEAD_DIM)
         k, v = synth.kv_chunk(3, 0, CHUNK, HEADS, HEAD_DIM, off)
         kd, vd = to_dev(k), to_dev(v)
         cache = nv.KVCache(HEADS, HEAD_DIM, CHUNK, WINDOW, dev)
         for sl in range(WINDOW):
             nv.kv_quant_append(cache, kd, vd, sl)
-        tq = 256
+        tq = SCORES_TQ
         q = to_dev(synth.activations(5, tq, HEADS * HEAD_DIM)).view(tq, HEADS, HEAD_DIM)
         s_out = torch.empty((HEADS, tq, WINDOW * CHUNK), dtype=torch.bfloat16, device=dev)
         fn = lambda: nv.kv_window_scores(cache, list(range(WINDOW)), [CHUNK] * WINDOW, q, 1.0, s_out)  # noqa: E731
