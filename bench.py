@@ -768,14 +768,28 @@ def run_single_kernel(args):
         cache = nv.KVCache(HEADS, HEAD_DIM, CHUNK, WINDOW, dev)
         for sl in range(WINDOW):
             nv.kv_quant_append(cache, kd, vd, sl)
-        tq = SCORES_TQ
+        tq = args.tq
         q = to_dev(synth.activations(5, tq, HEADS * HEAD_DIM)).view(tq, HEADS, HEAD_DIM)
         s_out = torch.empty((HEADS, tq, WINDOW * CHUNK), dtype=torch.bfloat16, device=dev)
-        fn = lambda: nv.kv_window_scores(cache, list(range(WINDOW)), [CHUNK] * WINDOW, q, 1.0, s_out)  # noqa: E731
+        win = list(range(WINDOW))
+        fn = lambda: nv.kv_window_scores(cache, win, [CHUNK] * WINDOW, q, 1.0, s_out)  # noqa: E731
+        # the same result through the window dequant to bf16 and a cuBLAS batched GEMM
+        ko = torch.empty((WINDOW * CHUNK, HEADS, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+        vo = torch.empty_like(ko)
+        s_pair = torch.empty_like(s_out)
+
+        def pair_fn():
+            nv.kv_dequant_window(cache, win, ko, vo)
+            torch.bmm(q.transpose(0, 1), ko.permute(1, 2, 0), out=s_pair)
         if args.kernel == "kv_context":
-            nv.kv_window_scores(cache, list(range(WINDOW)), [CHUNK] * WINDOW, q, 1.0 / 128.0, s_out)
+            nv.kv_window_scores(cache, win, [CHUNK] * WINDOW, q, 1.0 / 128.0, s_out)
             o = torch.empty((tq, HEADS, HEAD_DIM), dtype=torch.bfloat16, device=dev)
-            fn = lambda: nv.kv_window_context(cache, list(range(WINDOW)), [CHUNK] * WINDOW, s_out, o)  # noqa: E731
+            o_pair = torch.empty((HEADS, tq, HEAD_DIM), dtype=torch.bfloat16, device=dev)
+            fn = lambda: nv.kv_window_context(cache, win, [CHUNK] * WINDOW, s_out, o)  # noqa: E731
+
+            def pair_fn():
+                nv.kv_dequant_window(cache, win, ko, vo)
+                torch.bmm(s_out, vo.transpose(0, 1), out=o_pair)
     elif args.kernel in ("kv_append", "kv_window"):
         off = synth.kv_offsets(3, HEADS, HEAD_DIM)
         k, v = synth.kv_chunk(3, 0, CHUNK, HEADS, HEAD_DIM, off)
@@ -799,8 +813,19 @@ def run_single_kernel(args):
     e1.record()
     torch.cuda.synchronize()
     st = nv.get_device_status(0)
-    print(json.dumps({"kernel": args.kernel, "shape": args.shape, "iters": args.iters,
-                      "ms_per_call": e0.elapsed_time(e1) / args.iters, "status": st}))
+    line = {"kernel": args.kernel, "shape": args.shape, "iters": args.iters,
+            "ms_per_call": e0.elapsed_time(e1) / args.iters, "status": st}
+    if args.kernel in ("kv_scores", "kv_context"):
+        line["shape"] = f"{args.tq} queries x {HEADS} heads x {HEAD_DIM} against {WINDOW * CHUNK} keys"
+        for _ in range(args.kernel_warmup):
+            pair_fn()
+        e0.record()
+        for _ in range(args.iters):
+            pair_fn()
+        e1.record()
+        torch.cuda.synchronize()
+        line["window_then_bmm_ms"] = e0.elapsed_time(e1) / args.iters
+    print(json.dumps(line))
     if st != nv.OK:
         raise SystemExit(1)
 
@@ -844,6 +869,7 @@ def main():
                          "kv_scores | kv_context | lora_merge")
     ap.add_argument("--shape", default="8192,14336,3072", help="M,N,K for gemm; rows,cols for (de)quantize")
     ap.add_argument("--iters", type=int, default=3)
+    ap.add_argument("--tq", type=int, default=SCORES_TQ, help="queries for --kernel kv_scores / kv_context")
     ap.add_argument("--kernel-warmup", type=int, default=1,
                     help="untimed calls before the timed ones in --kernel mode")
     args = ap.parse_args()
