@@ -187,7 +187,11 @@ static __device__ __noinline__ uint32_t e2m1_index_exact_f64(float ax, float D) 
 // ~2^-20 of an E2M1 midpoint, ties included) take the exact comparison path.
 // Two-lane FP32 arithmetic (the .f32x2 forms of sm_100): each lane rounds to nearest
 // even exactly like the scalar operation, so a pair of results is bit-identical to two
-// scalar operations, at one instruction instead of two.
+// scalar operations, at one instruction instead of two.  A paired multiply whose result
+// feeds a paired add may still be contracted into one fused multiply-add by the
+// assembler (seen on sm_100a: a single rounding where two were written), so wherever the
+// intermediate rounding is part of the defined result, write the two steps with
+// __fmul_rn and __fadd_rn instead.
 __device__ __forceinline__ void mul2(float& d0, float& d1, float a0, float a1, float b0, float b1) {
   asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
       "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"

@@ -283,8 +283,9 @@ __device__ __forceinline__ float fmax_nan(float a, float b) {
 //   h = c / (1 + 2^x),  x = -2 u log2(e) = c (A c^2 + B),
 //   B = -2 sqrt(2/pi) log2(e), A = 0.044715 B,
 // with the hardware exp2 and reciprocal approximations (relative error ~2^-22 over
-// the binary32 range against the 2^-16 (|c| + |h|) the GEMM promises for h; large
-// |c| gives h = c or -0, infinities as the formula).
+// the binary32 range, inside the 2^-20 (|c| + |h|) the parity tests hold h to; large
+// |c| gives h = c or -0, infinities as the formula).  No paired multiply here feeds a
+// paired add, so no step can be contracted into a fused multiply-add.
 // Two values at a time: the FP32 steps as two-lane operations (same roundings as the
 // scalar form), exp2 and reciprocal per value.
 __device__ __forceinline__ void gelu_tanh2(float& c0, float& c1) {

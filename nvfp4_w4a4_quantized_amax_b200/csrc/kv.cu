@@ -31,7 +31,7 @@ namespace {
 constexpr int kStatsThreads = 256;   // 8 warps; each lane owns 8 consecutive columns
 constexpr int kStatsCols = 256;      // columns per CTA
 constexpr int kSplits = 64;          // most token splits of the stats pass (scratch size)
-constexpr int kStatsUnroll = 4;      // token rows in flight per warp
+constexpr int kStatsUnroll = 2;      // token rows in flight per warp (2, 4, 6, 8 measured: 2 fastest)
 constexpr int kMuThreads = 256;      // 8 warps share the splits of kMuCols columns
 constexpr int kMuCols = 32;
 constexpr int kEncThreads = 256;

@@ -301,10 +301,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int q = 0; q < 4; ++q) f16x2_to_f32x2(kh[q], ko[2 * q], ko[2 * q + 1]);  // e2m1 * s, exact
 #pragma unroll
-          for (int q = 0; q < 8; q += 2) {  // two roundings: the product, then the sum
-            mul2(ko[q], ko[q + 1], ko[q], ko[q + 1], gk, gk);
-            add2(ko[q], ko[q + 1], ko[q], ko[q + 1], mu[q], mu[q + 1]);
-          }
+          for (int q = 0; q < 8; ++q)  // two roundings: the product, then the sum
+            ko[q] = __fadd_rn(__fmul_rn(ko[q], gk), mu[q]);
           out = make_uint4(pack_bf16x2(ko[0], ko[1]), pack_bf16x2(ko[2], ko[3]), pack_bf16x2(ko[4], ko[5]),
                            pack_bf16x2(ko[6], ko[7]));
         }

@@ -224,6 +224,23 @@ def test_context_wrong_token_count_sets_shape_status(cuda_dev):
     assert torch.all(o == 0)  # its keys are read as zeros
 
 
+def test_many_tiny_slots_scores_and_context(cuda_dev):
+    """40 slots of 1..8 tokens listed out of order: every key tile straddles many slots
+    (the decoders' slot tracking, the per-slot g and mu); the output's 3 key tiles of
+    64 go to a cluster of three CTAs with an uneven row split."""
+    rng = np.random.default_rng(27)
+    fills = [int(x) for x in rng.integers(1, 9, size=40)]
+    cache, khat, vhat = build_cache(heads=3, chunk=8, fills=fills, seed=28, with_v=True)
+    order = [int(x) for x in rng.permutation(40)]
+    tokens = [fills[i] for i in order]
+    device_status(clear=True)
+    got, ref, bound, tk = run_scores(cache, khat, order, tokens, 150, 3, torch.float32, 0.125, 29)
+    assert_scores(got, ref, bound, tk)
+    got, ref, bound = run_context(cache, vhat, order, tokens, 150, 3, torch.float32, 30)
+    assert np.all(np.abs(got - ref) <= TOL * bound)
+    assert device_status() == nv.OK
+
+
 def test_attention_from_the_cache_end_to_end(cuda_dev):
     """scores -> softmax (torch, FP32, then bf16 weights) -> context, against attention in
     float64 on the oracle's K^ and V^: the bf16 weights bound the error (2^-8 of sum p|v|)."""
