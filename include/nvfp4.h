@@ -335,8 +335,11 @@ nvfp4_status kv_window_scores(const nvfp4_kv_cache* cache, const int32_t* slots_
 
 /* kv_window_context — the V side of attention from the NVFP4 cache: the weighted
  * sum of the window's values, O = P V^, with V dequantized inside the kernel (one
- * 128-key tile at a time, into shared memory; no bf16 copy of the window's V is
- * written).  [TW] §四, as for kv_window_scores.
+ * 64-key tile at a time, into shared memory; no bf16 copy of the window's V is
+ * written).  [TW] §四, as for kv_window_scores.  When few query tiles face many
+ * keys, the keys are split over the CTAs of a thread-block cluster (up to 8) and
+ * their FP32 partial sums are added in a fixed order, so the result does not depend
+ * on scheduling.
  *   slots_host, tokens_host, n_slots : the window (HOST arrays), Tk keys in list
  *              order, exactly as for kv_dequant_window_tokens.
  *   p        : device bf16 [heads][tq][ld_p] weights of the keys (e.g. the softmax
@@ -345,8 +348,9 @@ nvfp4_status kv_window_scores(const nvfp4_kv_cache* cache, const int32_t* slots_
  *   o_out    : device [tq][heads][head_dim] of ot (NVFP4_FP32 or NVFP4_BF16), row
  *              pitch ldo elements (>= heads * head_dim), base and pitch 16-byte aligned:
  *                O[i, h, d] = sum_j p[h, i, j] * V^[j, h, d],
- *              accumulated in FP32 by the tensor cores, V^ bit for bit the window's V
- *              that kv_dequant_window_tokens writes; bf16 output is the RNE of it.
+ *              accumulated in FP32 by the tensor cores (and FP32 adds of partial
+ *              sums), V^ bit for bit the window's V that kv_dequant_window_tokens
+ *              writes; bf16 output is the RNE of it.
  * Requires head_dim == 128.  A listed slot whose recorded token count differs sets
  * device status NVFP4_ERR_SHAPE (its keys then count as zero).  Errors:
  * INVALID_ARG, SHAPE, ALIGNMENT. */
