@@ -213,6 +213,20 @@ def test_context_keys_split_across_a_cluster(cuda_dev, heads, chunk, fills, slot
     assert device_status() == nv.OK
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_context_many_query_tiles_one_key_tile(cuda_dev, dtype):
+    """60 keys (one 64-key tile, so no key split) against 12763 queries of 4 heads: the
+    grid no longer fits one wave, so each CTA takes several query tiles (three; the last
+    group one, the last tile ragged) and writes its accumulators straight out."""
+    heads, tq = 4, 12763
+    cache, _, vhat = build_cache(heads=heads, chunk=64, fills=[60], seed=31, with_v=True)
+    device_status(clear=True)
+    got, ref, bound = run_context(cache, vhat, [0], [60], tq, heads, dtype, 32)
+    extra = 2.0 ** -8 * np.abs(ref) if dtype == torch.bfloat16 else 0.0
+    assert np.all(np.abs(got - ref) <= TOL * bound + extra)
+    assert device_status() == nv.OK
+
+
 def test_context_wrong_token_count_sets_shape_status(cuda_dev):
     cache, _, _ = build_cache(heads=1, chunk=2048, fills=[2048, 100], seed=25, with_v=True)
     p = torch.zeros((1, 8, 4096), dtype=torch.bfloat16, device="cuda")
