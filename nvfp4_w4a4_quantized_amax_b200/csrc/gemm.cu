@@ -38,9 +38,12 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tc.cuh"
 
 namespace nvfp4 {
 namespace {
+
+using namespace tc;
 
 constexpr int kBM = 128;           // tile rows (A rows, TMEM lanes)
 constexpr int kBN = 128;           // tile columns (W rows)
@@ -100,119 +103,12 @@ struct Params {
 };
 
 // ----------------------------------------------------------------- PTX helpers
-__device__ __forceinline__ uint32_t smem_u32(const void* p) {
-  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
-}
-
-__device__ __forceinline__ unsigned long long global_ns() {
-  unsigned long long t;
-  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
-  return t;
-}
-
-__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
-  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
-  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
-               : "memory");
-}
-
-__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
-  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(bar),
-               "r"(bytes)
-               : "memory");
-}
-
-// One poll: the thread is suspended until the phase completes or a 20 us hint
-// runs out (a poll loop without the hint measured 2-3 % slower GEMMs).
-__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, 20000;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// Bounded wait for the phase with `parity` to complete.  Returns false when the
-// wait gave up (time limit, or another role raised the abort flag).
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
-                                          unsigned long long limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0) {
-      if (*abort_flag) return false;
-      if (global_ns() - t0 > limit_ns) return false;
-    }
-  }
-}
-
-// Bounded wait that ignores the abort flag: used to drain this CTA's own
-// asynchronous copies and MMAs before it releases shared and tensor memory.
-__device__ __forceinline__ bool mbar_wait_drain(uint32_t bar, uint32_t parity, unsigned long long limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const unsigned long long t0 = global_ns();
-  for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if ((it & 63u) == 0 && global_ns() - t0 > limit_ns) return false;
-  }
-}
-
-__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint32_t bar,
-                                            int32_t x, int32_t y) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar), "r"(x), "r"(y)
-      : "memory");
-}
-
-// Tiled TMA store of a shared-memory box to global memory (coordinates are
-// element column x, row y; rows and columns outside the tensor are not written).
-__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, uint32_t src, int32_t x, int32_t y) {
-  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
-                   reinterpret_cast<uint64_t>(map)),
-               "r"(src), "r"(x), "r"(y)
-               : "memory");
-}
-
-__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint4 v) {
-  asm volatile("st.shared.v4.u32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
-               : "memory");
-}
-
+// (mbarriers with bounded waits, TMA tile loads and stores, descriptors: tc.cuh)
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
   asm volatile(
       "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
-}
-
-__device__ __forceinline__ void tc_fence_before() {
-  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
-}
-__device__ __forceinline__ void tc_fence_after() {
-  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
-}
-
-// Shared-memory matrix descriptor (tcgen05 format): start address, leading and
-// stride byte offsets (>> 4), descriptor version 1 at bits 46..47, layout type
-// at bits 61..63 (2 = 128-byte swizzle, 0 = no swizzle).
-__device__ __forceinline__ uint64_t smem_desc(uint32_t addr, uint32_t lbo, uint32_t sbo, uint32_t layout) {
-  uint64_t d = 0;
-  d |= (uint64_t)((addr >> 4) & 0x3FFFu);
-  d |= (uint64_t)((lbo >> 4) & 0x3FFFu) << 16;
-  d |= (uint64_t)((sbo >> 4) & 0x3FFFu) << 32;
-  d |= (uint64_t)1 << 46;
-  d |= (uint64_t)(layout & 7u) << 61;
-  return d;
 }
 
 // Instruction descriptor of kind::mxf4nvf4 with UE4M3 scales: A and B E2M1
@@ -341,9 +237,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  tc_fence_before();
+  fence_before();
   __syncthreads();
-  tc_fence_after();
+  fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // operands and scales were written by earlier kernels
   const unsigned long long limit = p.wait_limit_ns;
@@ -403,7 +299,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        tc_fence_after();
+        fence_after();
         const uint32_t d_tmem = tmem_base + a * kBN;
         for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
           const int s = it % kStages;
@@ -413,7 +309,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          tc_fence_after();
+          fence_after();
           const int nvalid = (int)min((int64_t)4, p.num_k64 - ks * 4);
           uint8_t* st = smem + s * kStageBytes;
           const uint32_t a_addr = smem_u32(st), b_addr = smem_u32(st + kABytes);
@@ -472,7 +368,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tmem_st_32x32b_x32(tmem_base + ((uint32_t)(quarter * 32) << 16) + kSfColBase + s * 32, r);
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        tc_fence_before();
+        fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(smem_u32(&sf_bar[s]));
       }
@@ -506,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
         break;
       }
-      tc_fence_after();
+      fence_after();
       const int64_t mt = tile % p.num_m, nt = tile / p.num_m;
       const int64_t row = mt * kBM + row_in_tile;
       const bool row_ok = row < p.M;
@@ -609,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               (uint16_t)(sc[0] | (sc[1] << 8));
         }
       }
-      tc_fence_before();
+      fence_before();
       mbar_arrive(smem_u32(&tempty_bar[a]));
     }
     if (p.q_amax_out) {
@@ -621,9 +517,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
 
-  tc_fence_before();
+  fence_before();
   __syncthreads();
-  tc_fence_after();
+  fence_after();
   if (warp == 0) {
     __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
@@ -834,9 +730,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
   }
-  tc_fence_before();
+  fence_before();
   cluster_sync();  // barriers of both CTAs initialized, tensor memory allocated
-  tc_fence_after();
+  fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();  // operands and scales were written by earlier kernels
   const unsigned long long limit = p.wait_limit_ns;
@@ -905,7 +801,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          tc_fence_after();
+          fence_after();
           const uint32_t d_tmem = tmem_base + a * kBN;
           for (int64_t ks = 0; ks < kstages; ++ks, ++it) {
             const int s = it % kStages;
@@ -914,7 +810,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
               ok = false;
               break;
             }
-            tc_fence_after();
+            fence_after();
             const int nvalid = (int)min((int64_t)4, p.num_k64 - ks * 4);
             uint8_t* st = smem + s * kStageBytes;
             const uint32_t a_addr = smem_u32(st), b_addr = smem_u32(st + kABytes);
@@ -987,7 +883,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
           }
         }
         asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-        tc_fence_before();
+        fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive_cluster(leader_sf_bar0 + (uint32_t)(s * 8));
       }
@@ -1035,12 +931,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
         *abort_flag = 1;
         break;
       }
-      tc_fence_after();
+      fence_after();
       uint32_t r[2][32];
       const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + a * kBN + cgroup * 64;
       tmem_ld_32x32b_x32(taddr, r[0]);
       tmem_ld_32x32b_x32(taddr + 32, r[1]);
-      tc_fence_before();
+      fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive_cluster(leader_tempty0 + (uint32_t)(a * 8));
       const int64_t mt = tile % p.num_m, nt = tile / p.num_m;
@@ -1158,9 +1054,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
 
-  tc_fence_before();
+  fence_before();
   cluster_sync();  // no CTA leaves while its peer may still use its shared or tensor memory
-  tc_fence_after();
+  fence_after();
   if (warp == 0) {
     __syncwarp();
     asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(512) : "memory");
