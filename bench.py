@@ -257,19 +257,24 @@ def run_ours(args, rank: int, world: int, local_rank: int):
         X2, A3, A3B, X5, KVK, KVV = inputs if inputs is not None else (
             x2, a3, a3b, x5, kvd[slot_counter[0] % 2][0], kvd[slot_counter[0] % 2][1])
         am = o.amax
-        timed("quantize_32768x3072", lambda: nv.nvfp4_quantize(X2, o.qx2, amax_out=am[0:1]), 3, events)
-        timed("dequantize_32768x3072", lambda: nv.nvfp4_dequantize(o.qx2, o.y2), 1, events)
+        # Order: a kernel inherits the dirty L2 lines of the one before it and pays for
+        # their write-back.  The memory-bound kernels with small outputs come first (each
+        # behind a small writer), the two big writers (dequantize 201 MB, KV window
+        # 403 MB) last among them, then the GEMMs, which read from L2 and leave DRAM
+        # time to spare for the write-back they inherit.
+        timed("quantize_8192x3072_ffn", lambda: nv.nvfp4_quantize(X5, o.qx5, amax_out=am[3:4]), 3, events)
         timed("quantize_8192x3072", lambda: nv.nvfp4_quantize(A3, o.qa3, amax_out=am[1:2]), 3, events)
-        timed("quantize_8192x14336", lambda: nv.nvfp4_quantize(A3B, o.qa3b, amax_out=am[2:3]), 3, events)
-        for i, (k, n) in enumerate(BLOCK_GEMMS):
-            a = o.qa3 if k == 3072 else o.qa3b
-            timed(f"gemm_{k}x{n}", lambda a=a, i=i: nv.nvfp4_gemm(a, wq[i], o.cs[i]), 1, events)
         slot = slot_counter[0] % SLOTS
         timed("kv_append_8192", lambda: nv.kv_quant_append(cache, KVK, KVV, slot), 4, events)
+        timed("quantize_8192x14336", lambda: nv.nvfp4_quantize(A3B, o.qa3b, amax_out=am[2:3]), 3, events)
+        timed("quantize_32768x3072", lambda: nv.nvfp4_quantize(X2, o.qx2, amax_out=am[0:1]), 3, events)
+        timed("dequantize_32768x3072", lambda: nv.nvfp4_dequantize(o.qx2, o.y2), 1, events)
         win = [(slot - WINDOW + 1 + j) % SLOTS for j in range(WINDOW)]
         timed("kv_window_4x8192", lambda: nv.kv_dequant_window(cache, win, o.ko, o.vo), 1, events)
         slot_counter[0] += 1
-        timed("quantize_8192x3072_ffn", lambda: nv.nvfp4_quantize(X5, o.qx5, amax_out=am[3:4]), 3, events)
+        for i, (k, n) in enumerate(BLOCK_GEMMS):
+            a = o.qa3 if k == 3072 else o.qa3b
+            timed(f"gemm_{k}x{n}", lambda a=a, i=i: nv.nvfp4_gemm(a, wq[i], o.cs[i]), 1, events)
         timed("gemm_ffn_up_gelu_requant", lambda: nv.nvfp4_gemm(o.qx5, q1, None, act=nv.ACT_GELU_TANH,
                                                                 q_out=o.qh, q_gscale_in=g_h,
                                                                 q_amax_out=am[6:7]), 2, events)
