@@ -351,9 +351,9 @@ nvfp4_status kv_window_scores(const nvfp4_kv_cache* cache, const int32_t* slots_
  *              accumulated in FP32 by the tensor cores (and FP32 adds of partial
  *              sums), V^ bit for bit the window's V that kv_dequant_window_tokens
  *              writes; bf16 output is the RNE of it.
- * Requires head_dim == 128.  A listed slot whose recorded token count differs sets
- * device status NVFP4_ERR_SHAPE (its keys then count as zero).  Errors:
- * INVALID_ARG, SHAPE, ALIGNMENT. */
+ * Requires head_dim == 128 and tq <= 65535 * 512.  A listed slot whose recorded token
+ * count differs sets device status NVFP4_ERR_SHAPE (its keys then count as zero).
+ * Errors: INVALID_ARG, SHAPE, ALIGNMENT. */
 nvfp4_status kv_window_context(const nvfp4_kv_cache* cache, const int32_t* slots_host, const int32_t* tokens_host,
                                int32_t n_slots, const void* p, int64_t tq, int64_t ld_p, void* o_out, int32_t ot,
                                int64_t ldo, nvfp4_stream_t stream);

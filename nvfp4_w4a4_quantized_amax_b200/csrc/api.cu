@@ -433,7 +433,8 @@ nvfp4_status kv_window_context(const nvfp4_kv_cache* cache, const int32_t* slots
   }
   const int64_t esz = ot == NVFP4_BF16 ? 2 : 4;
   if (tq < 0 || ld_p < total || ldo < (int64_t)cache->heads * 128) return NVFP4_ERR_SHAPE;
-  if (tq > (1ll << 31) || total > (1ll << 31) || (int64_t)cache->heads > 65535) return NVFP4_ERR_SHAPE;
+  // at most 65535 query groups of up to 4 query tiles of 128
+  if (tq > 65535ll * 4 * 128 || total > (1ll << 31) || (int64_t)cache->heads > 65535) return NVFP4_ERR_SHAPE;
   if (tq > 0 && (!aligned16(p) || (ld_p * 2) % 16 != 0)) return NVFP4_ERR_ALIGNMENT;
   if (!aligned16(o_out) || (ldo * esz) % 16 != 0) return NVFP4_ERR_ALIGNMENT;
   unsigned* status = nullptr;

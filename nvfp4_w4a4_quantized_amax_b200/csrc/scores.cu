@@ -1030,9 +1030,11 @@ cudaError_t launch_kv_context(const KVLayout& L, const int32_t* slots, const int
   // dequantization counted as half of one.  Ties keep the smaller S.
   const int64_t n_kt = (acc + kCtxKeys - 1) / kCtxKeys;
   const int64_t n_qt = (tq + kQ - 1) / kQ;
-  int best_g = 1, best_s = 1;
+  int best_g = (int)((n_qt + 65534) / 65535), best_s = 1;
   double best = -1.0;
-  for (int g = 1; g <= kCtxMaxG && g <= n_qt; ++g) {
+  const int64_t g_min = (n_qt + 65534) / 65535;  // grid.y (query groups) is at most 65535
+  if (g_min > kCtxMaxG) return cudaErrorInvalidValue;
+  for (int g = (int)g_min; g <= kCtxMaxG && g <= n_qt; ++g) {
     for (int sp = 1; sp <= kMaxSplit && sp <= n_kt; ++sp) {
       const int64_t conc = conc_cache[dev][sp].load(std::memory_order_relaxed);
       if (conc <= 0) continue;

@@ -200,3 +200,40 @@ def test_noalloc_cache_may_end_at_the_scratch_region():
     k = ctypes.c_void_p(4097)
     assert lib.kv_quant_append(ctypes.byref(h), k, k, 64, 0, None) == nv.ERR_INVALID_ARG
     assert lib.kv_quant_append_noalloc(ctypes.byref(h), k, k, 64, 0, None) == nv.ERR_ALIGNMENT
+
+
+def test_attention_side_host_checks():
+    """kv_window_scores / kv_window_context: head_dim, window, pitch, alignment and size
+    rules, each rejected on the host before the device lookup."""
+    lib = nv.library()
+    h = nv.nvfp4_kv_cache()
+    nbytes = ctypes.c_size_t()
+    assert lib.nvfp4_kv_cache_bytes(2, 128, 64, 2, ctypes.byref(nbytes)) == nv.OK
+    assert lib.nvfp4_kv_cache_init(ctypes.c_void_p(4096), nbytes.value, 2, 128, 64, 2, ctypes.byref(h)) == nv.OK
+    slots = (ctypes.c_int32 * 2)(0, 1)
+    toks = (ctypes.c_int32 * 2)(64, 30)                 # Tk = 94
+    p = ctypes.c_void_p(1 << 20)
+    S = lib.kv_window_scores
+    sc = ctypes.c_float(0.125)
+    ok_s = lambda tq=16, ldq=256, ld_s=96, out=p, st=nv.FP32, q=p, n=2, t=toks: S(  # noqa: E731
+        ctypes.byref(h), slots, t, n, q, tq, ldq, sc, out, st, ld_s, None)
+    assert ok_s(ld_s=92) == nv.ERR_SHAPE                           # ld_s < Tk
+    assert ok_s(ldq=200) == nv.ERR_SHAPE                           # ldq < heads * 128
+    assert ok_s(ld_s=98) == nv.ERR_ALIGNMENT                       # score rows not 16-byte multiples
+    assert ok_s(out=ctypes.c_void_p((1 << 20) + 4)) == nv.ERR_ALIGNMENT
+    assert ok_s(st=7) == nv.ERR_INVALID_ARG                        # output dtype
+    assert ok_s(n=0) == nv.ERR_INVALID_ARG                         # empty window
+    assert ok_s(t=(ctypes.c_int32 * 2)(64, 65)) == nv.ERR_SHAPE    # more tokens than a chunk holds
+    C = lib.kv_window_context
+    ok_c = lambda tq=16, ld_p=96, ldo=256, out=p, ot=nv.FP32: C(  # noqa: E731
+        ctypes.byref(h), slots, toks, 2, p, tq, ld_p, out, ot, ldo, None)
+    assert ok_c(ld_p=88) == nv.ERR_SHAPE                           # ld_p < Tk
+    assert ok_c(ldo=128) == nv.ERR_SHAPE                           # ldo < heads * 128
+    assert ok_c(ld_p=100) == nv.ERR_ALIGNMENT                      # weight rows not 16-byte multiples
+    assert ok_c(out=ctypes.c_void_p((1 << 20) + 8)) == nv.ERR_ALIGNMENT
+    assert ok_c(tq=65535 * 512 + 1) == nv.ERR_SHAPE                # more than 65535 groups of 4 query tiles
+    assert ok_c(tq=-1) == nv.ERR_SHAPE
+    h64 = nv.nvfp4_kv_cache()
+    assert lib.nvfp4_kv_cache_bytes(2, 64, 64, 2, ctypes.byref(nbytes)) == nv.OK
+    assert lib.nvfp4_kv_cache_init(ctypes.c_void_p(4096), nbytes.value, 2, 64, 64, 2, ctypes.byref(h64)) == nv.OK
+    assert C(ctypes.byref(h64), slots, toks, 2, p, 16, 96, p, nv.FP32, 128, None) == nv.ERR_SHAPE  # head_dim 64
