@@ -258,14 +258,15 @@ def run_ours(args, rank: int, world: int, local_rank: int):
             x2, a3, a3b, x5, kvd[slot_counter[0] % 2][0], kvd[slot_counter[0] % 2][1])
         am = o.amax
         # Order: a kernel inherits the dirty L2 lines of the one before it and pays for
-        # their write-back.  The memory-bound kernels with small outputs come first (each
-        # behind a small writer), the two big writers (dequantize 201 MB, KV window
-        # 403 MB) last among them, then the GEMMs, which read from L2 and leave DRAM
-        # time to spare for the write-back they inherit.
-        timed("quantize_8192x3072_ffn", lambda: nv.nvfp4_quantize(X5, o.qx5, amax_out=am[3:4]), 3, events)
-        timed("quantize_8192x3072", lambda: nv.nvfp4_quantize(A3, o.qa3, amax_out=am[1:2]), 3, events)
+        # their write-back.  The KV append, whose two passes are bound by latency and
+        # issue rather than DRAM, takes what the previous step's GEMMs left; the other
+        # memory-bound kernels with small outputs follow (each behind a small writer),
+        # the two big writers (dequantize 201 MB, KV window 403 MB) last among them, then
+        # the GEMMs, which read from L2 and leave DRAM time for the write-back they inherit.
         slot = slot_counter[0] % SLOTS
         timed("kv_append_8192", lambda: nv.kv_quant_append(cache, KVK, KVV, slot), 4, events)
+        timed("quantize_8192x3072_ffn", lambda: nv.nvfp4_quantize(X5, o.qx5, amax_out=am[3:4]), 3, events)
+        timed("quantize_8192x3072", lambda: nv.nvfp4_quantize(A3, o.qa3, amax_out=am[1:2]), 3, events)
         timed("quantize_8192x14336", lambda: nv.nvfp4_quantize(A3B, o.qa3b, amax_out=am[2:3]), 3, events)
         timed("quantize_32768x3072", lambda: nv.nvfp4_quantize(X2, o.qx2, amax_out=am[0:1]), 3, events)
         timed("dequantize_32768x3072", lambda: nv.nvfp4_dequantize(o.qx2, o.y2), 1, events)
