@@ -1,4 +1,4 @@
-// scores.cu — attention scores straight from the NVFP4 KV cache.
+// scores.cu — attention scores and outputs straight from the NVFP4 KV cache.
 //
 // techwalker.com, "NVIDIA研究团队打造全球首个FP4视频生成系统，速度提升两倍还省一半内存", §四:
 // K and V are kept in NVFP4 (K after subtracting its mean) and the chunks of the
@@ -15,7 +15,7 @@
 //                                                               writes)
 //
 // A persistent kernel (one CTA per SM) walks the (key tile, head) items; while one
-// item's query tiles go through the tensor cores and the epilogue, four warps decode
+// item's query tiles go through the tensor cores and the epilogue, six warps decode
 // the next item's keys into a second buffer.  The dequantized keys are reused by every
 // query tile, so the cache is read once per (head, key tile) and no bf16 copy of the
 // window exists in HBM.  The V side (P V^) follows below.
