@@ -146,9 +146,11 @@ __device__ __forceinline__ void encode_block(const EncodeParams& p, int64_t vb, 
   p.scales[soff] = (uint8_t)s;
 }
 
-// One thread encodes one 16-value block: block amax -> E4M3 scale -> 16 codes.
+// One thread encodes one 16-value block: block amax -> E4M3 scale -> 16 codes.  Six
+// resident CTAs per SM (40 registers, no spills): the pass is issue-bound, and 6
+// against 4 CTAs measured 3 % faster on 32768x3072 and 8192x14336 (7 and 8 spill).
 template <bool kBf16, bool kMma>
-__global__ void __launch_bounds__(kThreads) encode_kernel(EncodeParams p) {
+__global__ void __launch_bounds__(kThreads, 6) encode_kernel(EncodeParams p) {
   pdl_trigger();
   pdl_wait();
   float g;
