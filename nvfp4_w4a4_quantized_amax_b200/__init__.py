@@ -151,7 +151,32 @@ def _stream(stream):
 
 
 def _ptr(t) -> Optional[ctypes.c_void_p]:
-    return None if t is None else ctypes.c_void_p(t.data_ptr())
+    """Device address of a CUDA tensor (None stays NULL).  A host tensor is refused here:
+    its address would reach a kernel."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"a CUDA tensor is required, got one on {t.device}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _rows(t, name: str):
+    """t is [rows, cols] with unit stride along the row (the C calls take a row pitch);
+    an empty tensor's strides mean nothing and pass."""
+    if t.dim() != 2 or (t.numel() > 0 and t.shape[1] > 1 and t.stride(1) != 1):
+        raise ValueError(f"{name}: a 2-D tensor with contiguous rows is required")
+
+
+def _dense(t, name: str):
+    if t.numel() > 0 and not t.is_contiguous():
+        raise ValueError(f"{name}: a contiguous tensor is required")
+
+
+def _bf16(t, name: str):
+    import torch
+
+    if t.dtype != torch.bfloat16:
+        raise TypeError(f"{name}: bf16 is required, got {t.dtype}")
 
 
 def _dtype_code(t) -> int:
@@ -198,6 +223,7 @@ class NVFP4Tensor:
 
 def nvfp4_quantize(x, out: NVFP4Tensor, gscale_in=None, amax_out=None, stream=None):
     """Quantize x [rows, cols] (bf16 or fp32, CUDA) into `out`."""
+    _rows(x, "x")
     rows, cols = x.shape
     _check(library().nvfp4_quantize(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(gscale_in),
                                     ctypes.byref(out.c), _ptr(amax_out), _stream(stream)),
@@ -206,12 +232,14 @@ def nvfp4_quantize(x, out: NVFP4Tensor, gscale_in=None, amax_out=None, stream=No
 
 def nvfp4_amax(x, amax_out, stream=None):
     """max|x| of x [rows, cols] (bf16 or fp32, CUDA) into amax_out (fp32 [1], CUDA)."""
+    _rows(x, "x")
     rows, cols = x.shape
     _check(library().nvfp4_amax(_ptr(x), _dtype_code(x), rows, cols, x.stride(0), _ptr(amax_out),
                                 _stream(stream)), "nvfp4_amax")
 
 
 def nvfp4_dequantize(t: NVFP4Tensor, y, stream=None):
+    _rows(y, "y")
     _check(library().nvfp4_dequantize(ctypes.byref(t.c), _ptr(y), _dtype_code(y), y.stride(0),
                                       _stream(stream)), "nvfp4_dequantize")
 
@@ -224,6 +252,8 @@ def nvfp4_gemm(a: NVFP4Tensor, w: NVFP4Tensor, c=None, act: int = ACT_NONE,
     if act != ACT_NONE or q_out is not None or q_amax_out is not None or h_out is not None:
         ep = nvfp4_epilogue(act, 0, ctypes.pointer(q_out.c) if q_out is not None else None,
                             _ptr(q_gscale_in), _ptr(q_amax_out), _ptr(h_out))
+    if c is not None:
+        _rows(c, "c")
     ct = _dtype_code(c) if c is not None else FP32
     ldc = c.stride(0) if c is not None else 0
     _check(library().nvfp4_gemm(ctypes.byref(a.c), ctypes.byref(w.c), _ptr(c), ct, ldc,
@@ -283,6 +313,8 @@ class KVCache:
 def kv_quant_append(cache: KVCache, k, v, slot: int, stream=None):
     """Quantize one chunk (bf16 [tokens, heads, head_dim], 1 <= tokens <= chunk_tokens)
     of K and V into `slot`."""
+    _dense(k, "k")
+    _dense(v, "v")
     _check(library().kv_quant_append(ctypes.byref(cache.handle), _ptr(k), _ptr(v), k.shape[0], slot,
                                      _stream(stream)), "kv_quant_append")
 
@@ -292,11 +324,15 @@ def kv_quant_append_noalloc(cache: KVCache, k, v, slot: int, stream=None):
     per-device array holds the column statistics (heads * head_dim <= 4096).
     For callers that may not allocate device memory; calls racing on the GPU
     share that array, so issue them on one stream."""
+    _dense(k, "k")
+    _dense(v, "v")
     _check(library().kv_quant_append_noalloc(ctypes.byref(cache.handle), _ptr(k), _ptr(v), k.shape[0],
                                              slot, _stream(stream)), "kv_quant_append_noalloc")
 
 
 def kv_dequant_window(cache: KVCache, slots: Sequence[int], k_out, v_out, stream=None):
+    _dense(k_out, "k_out")
+    _dense(v_out, "v_out")
     arr = (ctypes.c_int32 * len(slots))(*slots)
     _check(library().kv_dequant_window(ctypes.byref(cache.handle), arr, len(slots), _ptr(k_out),
                                        _ptr(v_out), _stream(stream)), "kv_dequant_window")
@@ -307,6 +343,8 @@ def kv_dequant_window_tokens(cache: KVCache, slots: Sequence[int], tokens: Seque
     """Window over slots holding tokens[i] tokens each; output rows sum(tokens), in list order."""
     if len(tokens) != len(slots):
         raise ValueError("one token count per slot")
+    _dense(k_out, "k_out")
+    _dense(v_out, "v_out")
     sarr = (ctypes.c_int32 * len(slots))(*slots)
     tarr = (ctypes.c_int32 * len(tokens))(*tokens)
     _check(library().kv_dequant_window_tokens(ctypes.byref(cache.handle), sarr, tarr, len(slots), _ptr(k_out),
@@ -319,9 +357,15 @@ def kv_window_scores(cache: KVCache, slots: Sequence[int], tokens: Sequence[int]
     from the NVFP4 cache inside the kernel; s_out (fp32 or bf16 [heads, tq, >= Tk])."""
     if len(tokens) != len(slots):
         raise ValueError("one token count per slot")
+    _bf16(q, "q")
+    if q.dim() != 3 or q.shape[1] != cache.heads or (q.numel() > 0 and (q.stride(2) != 1 or q.stride(1) != q.shape[2])):
+        raise ValueError("q: [tq, heads, head_dim] with contiguous heads and dims is required")
+    tq = q.shape[0]
+    if s_out.dim() != 3 or s_out.shape[0] != cache.heads or s_out.shape[1] != tq or (
+            s_out.numel() > 0 and (s_out.stride(2) != 1 or s_out.stride(0) != tq * s_out.stride(1))):
+        raise ValueError("s_out: [heads, tq, ld_s] with rows ld_s apart and heads tq * ld_s apart is required")
     sarr = (ctypes.c_int32 * len(slots))(*slots)
     tarr = (ctypes.c_int32 * len(tokens))(*tokens)
-    tq = q.shape[0]
     _check(library().kv_window_scores(ctypes.byref(cache.handle), sarr, tarr, len(slots), _ptr(q), tq,
                                       q.stride(0), float(scale), _ptr(s_out), _dtype_code(s_out),
                                       s_out.stride(1), _stream(stream)), "kv_window_scores")
@@ -332,6 +376,13 @@ def kv_window_context(cache: KVCache, slots: Sequence[int], tokens: Sequence[int
     p bf16 [heads, tq, >= Tk]; o_out (fp32 or bf16) [tq, heads, head_dim]."""
     if len(tokens) != len(slots):
         raise ValueError("one token count per slot")
+    _bf16(p, "p")
+    if p.dim() != 3 or p.shape[0] != cache.heads or (
+            p.numel() > 0 and (p.stride(2) != 1 or p.stride(0) != p.shape[1] * p.stride(1))):
+        raise ValueError("p: [heads, tq, ld_p] with rows ld_p apart and heads tq * ld_p apart is required")
+    if o_out.dim() != 3 or o_out.shape[0] != p.shape[1] or o_out.shape[1] != cache.heads or (
+            o_out.numel() > 0 and (o_out.stride(2) != 1 or o_out.stride(1) != o_out.shape[2])):
+        raise ValueError("o_out: [tq, heads, head_dim] with contiguous heads and dims is required")
     sarr = (ctypes.c_int32 * len(slots))(*slots)
     tarr = (ctypes.c_int32 * len(tokens))(*tokens)
     _check(library().kv_window_context(ctypes.byref(cache.handle), sarr, tarr, len(slots), _ptr(p), p.shape[1],
@@ -343,6 +394,10 @@ def nvfp4_lora_merge(w, lora_b, lora_a, scale: float, out, stream=None):
     """out = W + scale * (B A) in binary32 with the library's fixed order (LoRA merged
     before quantization).  w: bf16 or fp32 [rows, cols]; lora_b fp32 [rows, rank];
     lora_a fp32 [rank, cols]; out fp32 [rows, cols]."""
+    _rows(w, "w")
+    _rows(out, "out")
+    _dense(lora_b, "lora_b")
+    _dense(lora_a, "lora_a")
     rows, cols = w.shape
     rank = lora_b.shape[1]
     _check(library().nvfp4_lora_merge(_ptr(w), _dtype_code(w), rows, cols, w.stride(0), _ptr(lora_b),

@@ -237,3 +237,19 @@ def test_attention_side_host_checks():
     assert lib.nvfp4_kv_cache_bytes(2, 64, 64, 2, ctypes.byref(nbytes)) == nv.OK
     assert lib.nvfp4_kv_cache_init(ctypes.c_void_p(4096), nbytes.value, 2, 64, 64, 2, ctypes.byref(h64)) == nv.OK
     assert C(ctypes.byref(h64), slots, toks, 2, p, 16, 96, p, nv.FP32, 128, None) == nv.ERR_SHAPE  # head_dim 64
+
+
+def test_binding_refuses_host_tensors_and_foreign_layouts():
+    """The Python binding passes device addresses only: a host tensor, or a layout the C
+    call cannot express with its row pitch, is refused before the library is called."""
+    import torch
+
+    x = torch.zeros(4, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        nv.nvfp4_amax(x, torch.zeros(1))
+    with pytest.raises(ValueError, match="CUDA"):
+        nv.nvfp4_lora_merge(torch.zeros(4, 32), torch.zeros(4, 2), torch.zeros(2, 32), 1.0, torch.zeros(4, 32))
+    with pytest.raises(ValueError, match="contiguous rows"):
+        nv.nvfp4_amax(x.t(), torch.zeros(1))
+    with pytest.raises(ValueError, match="contiguous"):
+        nv.nvfp4_lora_merge(torch.zeros(4, 32), torch.zeros(2, 4).t(), torch.zeros(2, 32), 1.0, torch.zeros(4, 32))
